@@ -1,0 +1,218 @@
+"""Pins for the oracle's exact attention and blockwise E4M3 emulator.
+
+What pins what:
+  * exact FP64 attention  <- PyTorch's scaled_dot_product_attention in float64
+    (a library routine), causal, non-causal and grouped-query;
+  * the online-softmax recurrence <- with the cast off it must reproduce the
+    exact attention to FP32 rounding (the re-association is exact in exact
+    arithmetic: "La ricorrenza softmax online");
+  * block order <- a single block gives identical results in both orders, and
+    the reverse order removes underflows outside the sink block;
+  * the scale S <- hand-checkable uniform-logit cases (P = 1 everywhere),
+    saturation at S = 512, and bit-identical outputs across S = 2^k when every
+    P is in the normal range;
+  * the underflow rule <- the per-row closed form of F(Delta, S) and the
+    threshold Delta_c of the P-cast summary (sections 2 and 3);
+  * the pages' measured magnitudes (section 4 and the lay explanation).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+from conftest import golden_facts
+
+FACTS = golden_facts()
+
+
+def rand_e4m3(rng, shape, scale=1.0):
+    x = (rng.standard_normal(shape) * scale).astype(np.float32)
+    return oracle.e4m3_encode(x)
+
+
+def torch_reference(q, k, v, causal):
+    qf, kf, vf = (torch.from_numpy(oracle.e4m3_decode(x).astype(np.float64)) for x in (q, k, v))
+    rep = qf.shape[1] // kf.shape[1]
+    kf, vf = kf.repeat_interleave(rep, 1), vf.repeat_interleave(rep, 1)
+    o = torch.nn.functional.scaled_dot_product_attention(qf, kf, vf, is_causal=causal)
+    s = qf @ kf.transpose(-1, -2) / math.sqrt(qf.shape[-1])
+    if causal:
+        n = s.shape[-1]
+        s = s.masked_fill(torch.triu(torch.ones(n, n, dtype=torch.bool), 1), float("-inf"))
+    return o.numpy(), torch.logsumexp(s, -1).numpy()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp64_matches_torch_sdpa(causal):
+    rng = np.random.default_rng(1)
+    q = rand_e4m3(rng, (2, 4, 77, 64), 2.0)
+    k = rand_e4m3(rng, (2, 2, 77, 64), 2.0)
+    v = rand_e4m3(rng, (2, 2, 77, 64))
+    o, lse = oracle.attention_fp64(q, k, v, causal)
+    o_ref, lse_ref = torch_reference(q, k, v, causal)
+    assert np.abs(o - o_ref).max() < 1e-12
+    assert np.abs(lse - lse_ref).max() < 1e-12
+    rows = np.array([0, 5, 76], dtype=np.int32)
+    o_s, lse_s = oracle.attention_fp64(q, k, v, causal, rows=rows)
+    assert np.array_equal(o_s, o[:, :, rows])
+    assert np.array_equal(lse_s, lse[:, :, rows])
+
+
+@pytest.mark.parametrize("causal,N,Bc,reverse", [
+    (False, 300, 64, False), (False, 300, 64, True), (True, 300, 64, False),
+    (True, 300, 64, True), (True, 512, 128, True), (False, 129, 128, False)])
+def test_emulator_without_cast_equals_exact(causal, N, Bc, reverse):
+    rng = np.random.default_rng(2)
+    q, k, v = rand_e4m3(rng, (1, 2, N, 64), 2.0), rand_e4m3(rng, (1, 2, N, 64), 2.0), rand_e4m3(rng, (1, 2, N, 64))
+    o64, lse64 = oracle.attention_fp64(q, k, v, causal)
+    for S in (1.0, 256.0):
+        r = oracle.emulate(q, k, v, causal=causal, block_n=Bc, p_scale=S, reverse=reverse, cast=False)
+        assert np.abs(r.o_f32 - o64).max() <= 1e-5 * np.abs(o64).max()
+        assert np.abs(r.lse - lse64).max() <= 1e-5 * max(1.0, np.abs(lse64).max())
+
+
+def test_single_block_is_order_independent():
+    rng = np.random.default_rng(3)
+    q, k, v = rand_e4m3(rng, (1, 3, 64, 64), 3.0), rand_e4m3(rng, (1, 3, 64, 64), 3.0), rand_e4m3(rng, (1, 3, 64, 64))
+    for causal in (False, True):
+        a = oracle.emulate(q, k, v, causal=causal, block_n=64, p_scale=1.0, reverse=False)
+        b = oracle.emulate(q, k, v, causal=causal, block_n=64, p_scale=1.0, reverse=True)
+        assert np.array_equal(a.o_bf16, b.o_bf16) and np.array_equal(a.lse, b.lse)
+        assert np.array_equal(a.zeros, b.zeros)
+
+
+@pytest.mark.parametrize("S,expected_factor", [(1.0, 1.0), (256.0, 1.0), (448.0, 1.0), (512.0, 448.0 / 512.0)])
+def test_uniform_logits(S, expected_factor):
+    # q = 0 makes every logit 0, so P = 1 for every key and P * S = S.  For
+    # S <= 448 the cast is exact and O is the mean of V; S = 512 saturates to
+    # 448 while the epilogue still divides by 512.
+    rng = np.random.default_rng(4)
+    N, d = 256, 64
+    q = np.zeros((1, 1, N, d), dtype=np.uint8)
+    k = rand_e4m3(rng, (1, 1, N, d))
+    v = rand_e4m3(rng, (1, 1, N, d))
+    r = oracle.emulate(q, k, v, causal=False, block_n=64, p_scale=S, reverse=False)
+    mean_v = oracle.e4m3_decode(v)[0, 0].astype(np.float64).mean(0)
+    assert np.allclose(r.o_f32[0, 0], expected_factor * mean_v[None, :], rtol=0, atol=1e-6)
+    assert r.zeros.sum() == 0
+
+
+def test_power_of_two_scales_agree_when_p_is_normal():
+    # Logits within +-1 keep every P >= e^-2 > 2^-6: the E4M3 cast then
+    # commutes with multiplication by 2^k (no subnormals, no saturation for
+    # S <= 256), so outputs are bit-identical across S = 1 .. 256.
+    rng = np.random.default_rng(5)
+    N, d = 512, 64
+    q = rand_e4m3(rng, (1, 2, N, d), 0.25)
+    k = rand_e4m3(rng, (1, 2, N, d), 0.25)
+    v = rand_e4m3(rng, (1, 2, N, d))
+    s = np.einsum("bhid,bhjd->bhij", *(oracle.e4m3_decode(x).astype(np.float64) for x in (q, k))) / 8.0
+    assert s.max() - s.min() < 2.0
+    ref = oracle.emulate(q, k, v, causal=False, block_n=64, p_scale=1.0, reverse=False)
+    for e in range(1, 9):
+        r = oracle.emulate(q, k, v, causal=False, block_n=64, p_scale=2.0 ** e, reverse=False)
+        assert np.array_equal(r.o_f32, ref.o_f32), e
+    r448 = oracle.emulate(q, k, v, causal=False, block_n=64, p_scale=448.0, reverse=False)
+    assert not np.array_equal(r448.o_f32, ref.o_f32)
+
+
+def test_cast_error_within_half_step_bound():
+    # Each cast value is within half an E4M3 step of P*S: relative 2^-4 in the
+    # normal range, 2^-10 absolute below it.  So per row and column
+    # |O_cast - O_nocast| <= sum_j (2^-4 w_j + 2^-10 / (S l)) |v_jc|, w the
+    # exact softmax weights and l >= 1 the denominator in units of the max.
+    rng = np.random.default_rng(6)
+    w = synthetic.WORKLOADS["tiny"]
+    q, k, v, _ = synthetic.workload_inputs(w, seed=1000)
+    qf, kf, vf = (oracle.e4m3_decode(x).astype(np.float64) for x in (q, k, v))
+    s = np.einsum("bhid,bhjd->bhij", qf, kf) / math.sqrt(w.d)
+    p = np.exp(s - s.max(-1, keepdims=True))
+    l = p.sum(-1, keepdims=True)
+    for S in (1.0, 256.0, 448.0):
+        for rev in (False, True):
+            a = oracle.emulate(q, k, v, causal=False, block_n=64, p_scale=S, reverse=rev)
+            b = oracle.emulate(q, k, v, causal=False, block_n=64, p_scale=S, reverse=rev, cast=False)
+            bound = np.einsum("bhij,bhjc->bhic", 2.0 ** -4 * p / l + 2.0 ** -10 / (S * l), np.abs(vf))
+            assert np.all(np.abs(a.o_f32 - b.o_f32) <= bound + 1e-6), (S, rev)
+
+
+def _row_stats(q, k, d):
+    qf, kf = (oracle.e4m3_decode(x).astype(np.float64) for x in (q, k))
+    s = np.einsum("bhid,bhjd->bhij", qf, kf) / math.sqrt(d)
+    return s.max(-1).ravel(), s[..., 4:].std(-1).ravel()
+
+
+@pytest.mark.parametrize("delta", [5.0, 6.0, 7.0, 8.0, 9.0])
+def test_forward_underflow_fraction_matches_closed_form(delta):
+    B, H, N, d = 1, 4, 2048, 128
+    q, k, v, _ = synthetic.make_inputs(B, H, H, N, d, delta, seed=77)
+    m, sig = _row_stats(q, k, d)
+    for S in (1.0, 4.0, 32.0):
+        r = oracle.emulate(q, k, v, causal=False, block_n=128, p_scale=S, reverse=False)
+        frac = r.zeros.sum() / r.eligible.sum()
+        assert abs(frac - oracle.f_row(m, sig, S)) <= 0.01, (delta, S, frac)
+
+
+def test_collapse_threshold_location():
+    B, H, N, d = 1, 4, 1024, 128
+    deltas = [4.0, 4.5, 5.0, 5.5, 6.0, 6.5, 7.0, 7.5, 8.0, 9.0, 10.0]  # all exact in E4M3
+    eff = 11.0 / math.sqrt(d)  # e4m3(sqrt(128)) = 11
+    for S in (1.0, 4.0):
+        frac = []
+        for delta in deltas:
+            q, k, v, _ = synthetic.make_inputs(B, H, H, N, d, delta, seed=88)
+            r = oracle.emulate(q, k, v, causal=False, block_n=128, p_scale=S, reverse=False)
+            frac.append(r.zeros.sum() / r.eligible.sum())
+        assert all(b >= a for a, b in zip(frac, frac[1:]))  # monotone in Delta
+        x = np.array(deltas) * eff
+        crossing = float(np.interp(0.5, np.array(frac), x))
+        assert abs(crossing - float(oracle.delta_c(S))) <= 0.25, (S, crossing)
+
+
+@pytest.mark.parametrize("delta", [7.0, 8.0])
+def test_reverse_order_with_s256_has_no_underflow_outside_sink_block(delta):
+    B, H, N, d = 1, 4, 4096, 128
+    q, k, v, _ = synthetic.make_inputs(B, H, H, N, d, delta, seed=99)
+    rev = oracle.emulate(q, k, v, causal=False, block_n=128, p_scale=256.0, reverse=True)
+    assert rev.zeros[..., 1].sum() == 0
+    fwd = oracle.emulate(q, k, v, causal=False, block_n=128, p_scale=1.0, reverse=False)
+    assert fwd.zeros[..., 1].sum() > 0.5 * fwd.eligible[..., 1].sum()
+
+
+def test_paper_magnitudes_at_n4096():
+    B, H, N, d = 1, 4, int(FACTS["experiment_n"]), 128
+    q, k, v, _ = synthetic.make_inputs(B, H, H, N, d, 7.0, seed=2000)
+    o64, _ = oracle.attention_fp64(q, k, v, False)
+
+    def mse(S, rev):
+        r = oracle.emulate(q, k, v, causal=False, block_n=128, p_scale=S, reverse=rev)
+        return float(np.mean((r.o.astype(np.float64) - o64) ** 2))
+
+    base, f256, f448, r256 = mse(1.0, False), mse(256.0, False), mse(448.0, False), mse(256.0, True)
+    # forward S=1 is 3-10x worse than the optimised configurations
+    for opt in (f256, r256):
+        assert FACTS["mse_ratio_fwd1_low"] <= base / opt <= FACTS["mse_ratio_fwd1_high"]
+    # forward S=256 below forward S=448 (the pages say by 10-15%; this
+    # construction gives a smaller gap, see the design notes)
+    assert f256 < f448
+    assert 0.02 <= 1.0 - f256 / f448 <= FACTS["mse_gain_256_vs_448_high"]
+    # saturation: reverse + 256 indistinguishable from forward + 256
+    assert abs(r256 / f256 - 1.0) <= 0.05
+
+
+def test_non_sink_mass_lost_at_sink_strength_7():
+    # v = 1 on non-sink keys and 0 on sinks: each output column is the
+    # non-sink probability mass that survives the cast (exact: FP64 attention).
+    B, H, N, d = 1, 4, int(FACTS["experiment_n"]), 128
+    q, k, v, _ = synthetic.make_inputs(B, H, H, N, d, 7.0, seed=2000, v_mode="mass")
+    o64, _ = oracle.attention_fp64(q, k, v, False)
+    r = oracle.emulate(q, k, v, causal=False, block_n=128, p_scale=1.0, reverse=False)
+    per_row = 1.0 - (r.o_f32[..., 0] / o64[..., 0]).mean()
+    pooled = 1.0 - r.o_f32[..., 0].sum() / o64[..., 0].sum()
+    for loss in (per_row, pooled):
+        assert FACTS["non_sink_loss_low"] <= loss <= FACTS["non_sink_loss_high"], loss
+    r256 = oracle.emulate(q, k, v, causal=False, block_n=128, p_scale=256.0, reverse=True)
+    assert abs(1.0 - r256.o_f32[..., 0].sum() / o64[..., 0].sum()) < 0.01
