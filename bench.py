@@ -1,0 +1,355 @@
+"""Throughput benchmark of the FP8 (E4M3) P-cast attention forward pass.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one forward pass of the 32K causal prefill (B=1, H=32, N=32768,
+d=128, Delta=7 sink with k=4, S=256, reverse KV order) through the C ABI.
+Rank 0 prints one JSON line (see the design doc for every key).  Under torchrun
+each rank runs its own copy of the workload on its own GPU (no collective on
+the data path: weak scaling); the step time is the maximum over ranks.
+
+--impl reference times the CPU oracle (the blockwise E4M3 emulator) on the
+host cores instead, on a bounded sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synthetic  # noqa: E402
+
+WORKLOAD = synthetic.WORKLOADS["prefill32k"]
+P_SCALE = 256.0
+KV_ORDER = 1  # reverse
+SEED = 3000
+METRIC = "FP8 attn fwd TFLOP/s (% of FP8 peak) at N=32K,d=128; output MSE vs FP64"
+UNIT = "TFLOP/s"
+WORKLOAD_DESC = ("prefill32k: B=1 H=32 N=32768 d=128 causal, E4M3 Q/K/V, Delta=7 sink (k=4), S=256, "
+                 "reverse KV order")
+KERNEL_NAME = "fwd_v1_kernel"
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fwd_prefill32k_traffic.json")
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_BF16_TFLOPS = 1590.0
+FP8_OVER_BF16 = 2.0  # nominal dense ratio: 4.5 PF FP8 / 2.25 PF BF16
+CPU_SAMPLE_ROWS = 2048  # query rows per head the oracle arm evaluates per step
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--skip-cpu-baseline", action="store_true",
+                    help="omit the oracle timing (used under ncu)")
+    return ap.parse_args()
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "softmax_cast_precision_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as fh:
+            h.update(name.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def fp8_peak():
+    """FP8 dense peak: the measured BF16 cuBLAS figure x the nominal FP8/BF16 ratio."""
+    try:
+        with open(PEAKS_FILE) as fh:
+            pk = json.load(fh)
+        return pk["bf16_tflops"] * FP8_OVER_BF16, pk["bf16_tflops_sustained"] * FP8_OVER_BF16, "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_BF16_TFLOPS * FP8_OVER_BF16, 1400.0 * FP8_OVER_BF16, "fallback"
+
+
+def traffic_per_launch():
+    """DRAM bytes per launch from the committed ncu summary, if it is for this kernel source."""
+    try:
+        with open(PROFILE_SUMMARY) as fh:
+            s = json.load(fh)
+    except (OSError, ValueError):
+        return None
+    if s.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return s.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                clk, mx = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            sm.append(clk)
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        loaded = [c for c in sm if c > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def sample_rows(N: int, count: int) -> np.ndarray:
+    return synthetic.sampled_rows(N, count)
+
+
+def visible_pairs(rows: np.ndarray, N: int, causal: bool) -> int:
+    return int(np.sum(rows + 1)) if causal else int(len(rows) * N)
+
+
+def cpu_oracle_run(q, k, v, rows):
+    """One bounded step of the oracle arm: the emulator on `rows` of every head."""
+    import oracle
+
+    w = WORKLOAD
+    t0 = time.perf_counter()
+    oracle.emulate(q, k, v, causal=w.causal, block_n=128, p_scale=P_SCALE, reverse=bool(KV_ORDER), rows=rows)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * w.d * visible_pairs(rows, w.N, w.causal) * w.B * w.H
+    return flops, dt
+
+
+def cpu_baseline(q, k, v):
+    import oracle
+
+    rows = sample_rows(WORKLOAD.N, CPU_SAMPLE_ROWS)
+    flops, dt = cpu_oracle_run(q, k, v, rows)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"blockwise E4M3 emulator on {len(rows)} evenly spaced query rows of each of the "
+                      f"{WORKLOAD.B * WORKLOAD.H} heads ({flops / 1e12:.3f} TFLOP in {dt:.1f} s)"}
+
+
+def mse_vs_fp64(qd, kd, vd, o, rows_np):
+    """MSE of the output against exact attention computed in FP64 by PyTorch on
+    the same decoded E4M3 inputs, over the given query rows of every head."""
+    import torch
+
+    w = WORKLOAD
+    rows = torch.from_numpy(rows_np.astype(np.int64)).to(qd.device)
+    qf = qd.view(torch.float8_e4m3fn)[:, :, rows].double()
+    kf = kd.view(torch.float8_e4m3fn).double()
+    vf = vd.view(torch.float8_e4m3fn).double()
+    rep = w.H // w.Hkv
+    kf, vf = kf.repeat_interleave(rep, 1), vf.repeat_interleave(rep, 1)
+    s = qf @ kf.transpose(-1, -2) / math.sqrt(w.d)
+    if w.causal:
+        keys = torch.arange(w.N, device=qd.device)
+        s = s.masked_fill(keys[None, None, None, :] > rows[None, None, :, None], float("-inf"))
+    ref = torch.softmax(s, -1) @ vf
+    return float(((o[:, :, rows].double() - ref) ** 2).mean().item())
+
+
+def run_reference(args, rank, world):
+    """The oracle arm: emulator steps on the host cores (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle
+
+    q, k, v, _ = synthetic.workload_inputs(WORKLOAD, seed=SEED)
+    rows = sample_rows(WORKLOAD.N, 128)
+    for _ in range(args.warmup):
+        cpu_oracle_run(q, k, v, rows[:8])
+    total_flops, total_t = 0.0, 0.0
+    for _ in range(args.steps):
+        f, dt = cpu_oracle_run(q, k, v, rows)
+        total_flops += f
+        total_t += dt
+    value = total_flops / total_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3/f32",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_DESC, "l2": "inputs exceed L2"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"per step: the emulator on {len(rows)} evenly spaced query rows of each head"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+
+    from softmax_cast_precision_b200 import fp8attn
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+
+    w = WORKLOAD
+    q, k, v, _ = synthetic.workload_inputs(w, seed=SEED + rank)
+    qd, kd, vd = (torch.from_numpy(x).to(device) for x in (q, k, v))
+    o = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        fp8attn.fwd(qd, kd, vd, causal=w.causal, p_scale=P_SCALE, kv_order=KV_ORDER, out=o, lse_out=lse,
+                    stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    fp8attn.check_error(stream=stream, device=device)
+
+    # --- device-timed region: K steps, one kernel launch each --------------
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize(device)
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+    fp8attn.check_error(stream=stream, device=device)
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = ev[0].elapsed_time(ev[-1])
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    flops = w.flops()
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # --- end to end through the public API with host buffers ----------------
+    qh, kh, vh = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
+    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    e2e_steps = max(3, min(args.steps, 10))
+    fp8attn.fwd(qh, kh, vh, causal=w.causal, p_scale=P_SCALE, kv_order=KV_ORDER, out=oh, lse_out=lh,
+                device=device)
+    barrier()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        fp8attn.fwd(qh, kh, vh, causal=w.causal, p_scale=P_SCALE, kv_order=KV_ORDER, out=oh, lse_out=lh,
+                    device=device)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+    h2d = q.nbytes + k.nbytes + v.nbytes
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+
+    mse = mse_vs_fp64(qd, kd, vd, o, sample_rows(w.N, 256)) if rank == 0 else None
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peak_burst, peak_sustained, peak_src = fp8_peak()
+    kernel_ms = statistics.mean(per_step)
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    traffic = traffic_per_launch()
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_DESC, "flop_per_step_per_gpu": flops, "l2": "inputs exceed L2 (402 MB)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_burst, "unit": "TFLOP/s",
+                     "frac": achieved / peak_burst, "traffic": traffic,
+                     "peak_source": f"{peak_src}: bf16 cuBLAS burst x {FP8_OVER_BF16} (FP8/BF16 nominal)",
+                     "frac_of_sustained": achieved / peak_sustained},
+        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "clocks": clk.summary(),
+        "mse_vs_fp64": {"value": mse, "rows": "256 evenly spaced query rows of each head",
+                        "reference": "PyTorch float64 softmax(QK^T/sqrt(d))V on the same E4M3 inputs"},
+    }
+    if not args.skip_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(q, k, v)
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

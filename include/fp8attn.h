@@ -1,0 +1,107 @@
+/*
+ * fp8attn.h -- C ABI of libfp8attn: FP8 (E4M3) attention forward pass on
+ * NVIDIA B200 (sm_100a) with a static P-cast scale.
+ *
+ * The operation (the page "P-Cast Precision in FP8 Attention: Sink-Induced
+ * Collapse and the Optimality of S=2^8", technical summary, section 1):
+ * blockwise online-softmax attention O = softmax(Q K^T / sqrt(d)) V in which
+ * each probability tile P is multiplied by a static scale S, cast to E4M3
+ * before the P V product, and S is divided back out in the epilogue; the KV
+ * blocks are walked forward (block 0 first) or in reverse (last block first).
+ * The blockwise algorithm and its online-softmax recurrence are those of the
+ * page "Attenzione flash e domanda sulla lunghezza della sequenza", sections
+ * "L'algoritmo Flash Attention" and "La ricorrenza softmax online"; causal
+ * block skipping is its section on causal masking.
+ *
+ * Conventions shared by every call:
+ *   - All tensor arguments are DEVICE pointers to caller-owned memory; the
+ *     library keeps no pointer after a call returns and allocates no device
+ *     memory.  Pointers must be 16-byte aligned.
+ *   - Layouts are contiguous, row-major, with the head dimension innermost:
+ *       q    [B, H,   N, d]  E4M3 bytes (OCP E4M3FN)
+ *       k, v [B, Hkv, N, d]  E4M3 bytes
+ *       o    [B, H,   N, d]  bfloat16
+ *       lse  [B, H,   N]     float32
+ *     Query head h reads key/value head h / (H / Hkv) (grouped-query
+ *     attention; Hkv == H is ordinary multi-head attention).
+ *   - d must be 64 or 128.  N >= 0 is arbitrary (a ragged last tile is
+ *     masked).  B * H * N == 0 is a valid empty problem: nothing is launched.
+ *   - causal != 0 applies the square, top-left aligned mask (query i sees keys
+ *     0..i); KV blocks entirely above the diagonal are skipped.
+ *   - The logit scale is fixed at 1/sqrt(d).
+ *   - p_scale is the static scale S (finite, > 0).  Powers of two make the
+ *     scaling exact in FP32; S > 448 saturates the largest probabilities.
+ *   - kv_order: 0 = forward (KV block 0 first), 1 = reverse (last block
+ *     first).
+ *   - stream is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous with respect to the host: a return of
+ *     FP8ATTN_OK means the arguments were valid and the launch succeeded.
+ *   - On any error nothing is launched and outputs are left untouched; the
+ *     library never aborts the process and never traps on the device.
+ *   - Device-side waits are bounded.  A wait that runs out sets a device
+ *     error word instead of hanging; fp8attn_check_error() reports it.
+ */
+#ifndef FP8ATTN_H
+#define FP8ATTN_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every call. */
+enum fp8attn_status {
+    FP8ATTN_OK = 0,
+    FP8ATTN_ERR_INVALID_ARG = 1, /* a size, pointer, alignment or scale is invalid */
+    FP8ATTN_ERR_UNSUPPORTED = 2, /* valid but not supported here (d, device)       */
+    FP8ATTN_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed            */
+    FP8ATTN_ERR_TIMEOUT = 4      /* a device-side bounded wait ran out              */
+};
+
+/*
+ * Forward pass.  Writes o (bfloat16, O = sum_j P^_j v_j / (S * l)) and, when
+ * lse is not NULL, lse = m + ln(l): the natural log of the softmax
+ * denominator in units of the scaled logits q.k/sqrt(d), l being the sum of
+ * the unquantised probabilities.
+ */
+int fp8attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                int B, int H, int Hkv, int N, int d, int causal,
+                float p_scale, int kv_order, void* stream);
+
+/*
+ * P-collapse count.  Runs the same forward pass (same tiles, order, scale and
+ * cast) without writing O, and writes counts[b * H + h] = the number of
+ * (query, key) pairs of head (b, h) with key index j >= n_sink, not masked,
+ * whose cast value E4M3(P * S) is zero.  counts is a device array of B * H
+ * unsigned 64-bit integers; it is overwritten.  n_sink >= 0.  (Underflow of
+ * non-sink probabilities to zero is the "P-collapse" of the P-cast summary,
+ * section 1; passing n_sink equal to fp8attn_kv_tile(d) counts only keys
+ * outside the block that holds the sinks.)
+ */
+int fp8attn_pzero_count(const void* q, const void* k, const void* v,
+                        unsigned long long* counts,
+                        int B, int H, int Hkv, int N, int d, int causal,
+                        float p_scale, int kv_order, int n_sink, void* stream);
+
+/* KV block size B_c the kernels use for head dimension d (0 if d is
+ * unsupported).  The query block is always 128 rows. */
+int fp8attn_kv_tile(int d);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fp8attn_status_str(int status);
+
+/*
+ * Synchronises stream, then reads and clears the device error word that
+ * bounded waits set.  Returns FP8ATTN_ERR_TIMEOUT if a wait ran out since the
+ * last check, FP8ATTN_ERR_CUDA if the synchronisation itself failed, else
+ * FP8ATTN_OK.
+ */
+int fp8attn_check_error(void* stream);
+
+/* Library version as an integer (major * 10000 + minor * 100 + patch). */
+int fp8attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8ATTN_H */

@@ -1,0 +1,218 @@
+// api.cu -- the C ABI of libfp8attn (declared in include/fp8attn.h): argument
+// validation, TMA tensor-map construction and kernel launch.  No allocation:
+// every tensor is caller-owned device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fp8attn.h"
+#include "fwd_v1.cuh"
+#include "fwd_v2.cuh"
+
+namespace fp8attn {
+
+// Device error word set by bounded waits that run out (one per process and
+// device image; read and cleared by fp8attn_check_error).
+__device__ uint32_t g_error_word;
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// A [Z, rows, D] byte tensor (D contiguous) read in boxes of box_rows x D,
+// swizzled so that the tile lands in the layout the tcgen05 descriptors
+// describe (128-byte swizzle for 128-byte rows, 64-byte for 64-byte rows).
+bool make_map(CUtensorMap* map, const void* ptr, int D, int rows, int Z, int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(Z)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(D) * static_cast<cuuint64_t>(rows)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUtensorMapSwizzle swz = (D == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int validate(const void* q, const void* k, const void* v, int B, int H, int Hkv, int N, int d, float p_scale,
+             int kv_order) {
+  if (B < 0 || N < 0 || H < 1 || Hkv < 1 || H % Hkv != 0) return FP8ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FP8ATTN_ERR_UNSUPPORTED;
+  if (!(p_scale > 0.0f) || !std::isfinite(p_scale)) return FP8ATTN_ERR_INVALID_ARG;
+  if (kv_order != 0 && kv_order != 1) return FP8ATTN_ERR_INVALID_ARG;
+  if (B > 65535 || H > 65535) return FP8ATTN_ERR_UNSUPPORTED;  // grid y/z limits
+  const int64_t zq = static_cast<int64_t>(B) * H;
+  if (zq * N > (int64_t(1) << 40)) return FP8ATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * N * H == 0) return FP8ATTN_OK;
+  if (!q || !k || !v || !aligned16(q) || !aligned16(k) || !aligned16(v)) return FP8ATTN_ERR_INVALID_ARG;
+  return FP8ATTN_OK;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+// Persistent warp-specialised kernel (d = 128): one CTA per SM.
+template <bool COUNT>
+int launch_v2(const void* q, const void* k, const void* v, FwdParams p, cudaStream_t stream) {
+  using C = V2Config;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, 128, p.N, p.B * p.H, 128) || !make_map(&tk, k, 128, p.N, p.B * p.Hkv, 128) ||
+      !make_map(&tv, v, 128, p.N, p.B * p.Hkv, 128))
+    return FP8ATTN_ERR_CUDA;
+  auto kern = fwd_v2_kernel<COUNT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return FP8ATTN_ERR_CUDA;
+  // The warpgroups re-split the block's registers with setmaxnreg; that split
+  // is only valid for the launch register count it was computed for.
+  cudaFuncAttributes attr;
+  if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) return FP8ATTN_ERR_CUDA;
+  if (attr.numRegs != C::LAUNCH_REGS) return FP8ATTN_ERR_UNSUPPORTED;
+  uint32_t* err_word = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err_word), g_error_word) != cudaSuccess)
+    return FP8ATTN_ERR_CUDA;
+  const int sms = num_sms();
+  if (sms <= 0) return FP8ATTN_ERR_CUDA;
+  p.num_q_tiles = (p.N + 127) / 128;
+  p.num_kv_tiles = (p.N + 127) / 128;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
+  const int64_t units = static_cast<int64_t>(p.B) * p.H * ((p.N + 255) / 256);
+  const int grid = static_cast<int>(units < sms ? units : sms);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p, err_word);
+  return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
+}
+
+template <int D, bool COUNT>
+int launch(const void* q, const void* k, const void* v, FwdParams p, cudaStream_t stream) {
+  using C = V1Config<D>;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, D, p.N, p.B * p.H, C::BM) || !make_map(&tk, k, D, p.N, p.B * p.Hkv, C::BN) ||
+      !make_map(&tv, v, D, p.N, p.B * p.Hkv, C::BN))
+    return FP8ATTN_ERR_CUDA;
+  auto kern = fwd_v1_kernel<D, COUNT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return FP8ATTN_ERR_CUDA;
+  uint32_t* err_word = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err_word), g_error_word) != cudaSuccess)
+    return FP8ATTN_ERR_CUDA;
+  p.num_q_tiles = (p.N + C::BM - 1) / C::BM;
+  p.num_kv_tiles = (p.N + C::BN - 1) / C::BN;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+  dim3 grid(p.num_q_tiles, p.H, p.B);
+  kern<<<grid, 128, C::SMEM_BYTES, stream>>>(tq, tk, tv, p, err_word);
+  return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
+}
+
+FwdParams base_params(int B, int H, int Hkv, int N, int causal, float p_scale, int kv_order) {
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.h_per_kv = H / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.reverse = kv_order;
+  p.p_scale = p_scale;
+  return p;
+}
+
+}  // namespace
+}  // namespace fp8attn
+
+using namespace fp8attn;
+
+extern "C" int fp8attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Hkv,
+                           int N, int d, int causal, float p_scale, int kv_order, void* stream) {
+  int st = validate(q, k, v, B, H, Hkv, N, d, p_scale, kv_order);
+  if (st != FP8ATTN_OK) return st;
+  if (static_cast<int64_t>(B) * H * N == 0) return FP8ATTN_OK;
+  if (!o || !aligned16(o) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))) return FP8ATTN_ERR_INVALID_ARG;
+  FwdParams p = base_params(B, H, Hkv, N, causal, p_scale, kv_order);
+  p.o = o;
+  p.lse = lse;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 128 ? launch_v2<false>(q, k, v, p, s) : launch<64, false>(q, k, v, p, s);
+}
+
+extern "C" int fp8attn_pzero_count(const void* q, const void* k, const void* v, unsigned long long* counts, int B,
+                                   int H, int Hkv, int N, int d, int causal, float p_scale, int kv_order, int n_sink,
+                                   void* stream) {
+  int st = validate(q, k, v, B, H, Hkv, N, d, p_scale, kv_order);
+  if (st != FP8ATTN_OK) return st;
+  if (n_sink < 0) return FP8ATTN_ERR_INVALID_ARG;
+  const int64_t nheads = static_cast<int64_t>(B) * H;
+  if (nheads == 0) return FP8ATTN_OK;
+  if (!counts || (reinterpret_cast<uintptr_t>(counts) & 7u)) return FP8ATTN_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(counts, 0, sizeof(unsigned long long) * nheads, s) != cudaSuccess) return FP8ATTN_ERR_CUDA;
+  if (N == 0) return FP8ATTN_OK;
+  FwdParams p = base_params(B, H, Hkv, N, causal, p_scale, kv_order);
+  p.counts = counts;
+  p.n_sink = n_sink;
+  return d == 128 ? launch_v2<true>(q, k, v, p, s) : launch<64, true>(q, k, v, p, s);
+}
+
+extern "C" int fp8attn_kv_tile(int d) {
+  if (d == 128) return V1Config<128>::BN;
+  if (d == 64) return V1Config<64>::BN;
+  return 0;
+}
+
+extern "C" const char* fp8attn_status_str(int status) {
+  switch (status) {
+    case FP8ATTN_OK:
+      return "ok";
+    case FP8ATTN_ERR_INVALID_ARG:
+      return "invalid argument";
+    case FP8ATTN_ERR_UNSUPPORTED:
+      return "unsupported configuration";
+    case FP8ATTN_ERR_CUDA:
+      return "CUDA error";
+    case FP8ATTN_ERR_TIMEOUT:
+      return "device wait timed out";
+    default:
+      return "unknown status";
+  }
+}
+
+extern "C" int fp8attn_check_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FP8ATTN_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return FP8ATTN_ERR_CUDA;
+  if (word != 0) {
+    const uint32_t zero = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return FP8ATTN_ERR_CUDA;
+    return FP8ATTN_ERR_TIMEOUT;
+  }
+  return FP8ATTN_OK;
+}
+
+extern "C" int fp8attn_version(void) { return 100; }

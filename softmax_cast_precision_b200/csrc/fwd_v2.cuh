@@ -1,0 +1,468 @@
+// fwd_v2.cuh -- persistent, warp-specialised sm_100a forward kernel (d = 128).
+//
+// One CTA per SM walks a static, heaviest-first list of work units; a unit is
+// a pair of adjacent 128-row query tiles (Q0, Q1) of one (batch, head).  Roles:
+//   warps 0-3  softmax for Q0  (TMEM lanes 0..127 of S0 and O0)
+//   warps 4-7  softmax for Q1  (TMEM lanes 0..127 of S1 and O1)
+//   warp  8    TMA producer: Q pair per unit, K and V tiles through a ring
+//   warp  9    MMA issuer: S_k = Q_k K^T and O_k += P^_k V (tcgen05, FP8 E4M3),
+//              and owner of the tensor-memory allocation
+//   warps 10-11 idle (they complete the producer warpgroup for setmaxnreg)
+// Tensor memory: S0 cols [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+// The two softmax warpgroups alternate on the tensor core: while one turns
+// its S tile into P^, the MMA warp runs the other's products, so the tensor
+// core and the exponential/convert pipes overlap.
+//
+// Per KV tile and query row the arithmetic is that of the simple kernel:
+// running max over every block, P = 2^(x - m), l from unquantised P, the
+// P-cast E4M3(P * S), exact retroactive rescale of O when the max grew, and
+// O / (S * l) at the end ("P-Cast Precision in FP8 Attention", technical
+// summary, section 1; "Attenzione flash e domanda sulla lunghezza della
+// sequenza", sections "L'algoritmo Flash Attention" and the causal-masking
+// section).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "fwd_v1.cuh"
+#include "sm100_ptx.cuh"
+
+namespace fp8attn {
+
+struct V2Config {
+  static constexpr int D = 128;
+  static constexpr int BM = 128;
+  static constexpr int BN = 128;
+  static constexpr int STAGES = 3;
+  static constexpr int TILE_BYTES = 128 * 128;  // one 128 x 128 E4M3 tile
+  static constexpr int OFF_Q = 0;                               // Q0, Q1
+  static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;          // K ring
+  static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;     // V ring
+  static constexpr int OFF_P = OFF_V + STAGES * TILE_BYTES;     // P0 x2, P1 x2 (double-buffered)
+  static constexpr int OFF_BAR = OFF_P + 4 * TILE_BYTES;
+  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // control block + alignment slack
+  static constexpr int THREADS = 384;  // 3 warpgroups
+  // Register split (setmaxnreg): the block launches with 168 registers per
+  // thread (65536 / 384 rounded down to a multiple of 8); the producer
+  // warpgroup gives registers back and the two softmax warpgroups take them.
+  static constexpr int LAUNCH_REGS = 168;
+  static constexpr int SOFTMAX_REGS = 224;
+  static constexpr int PRODUCER_REGS = 56;
+  static constexpr uint32_t TMEM_COLS = 512;
+};
+
+// Shared-memory control block.
+struct V2Bars {
+  uint64_t q_full, q_empty;
+  uint64_t k_full[V2Config::STAGES], v_full[V2Config::STAGES], kv_empty[V2Config::STAGES];
+  uint64_t s_full[2], s_free[2], p_full[2], o_done[2], o_free[2];
+  uint64_t drain;  // MMA warp: all issued tensor-core work complete
+  uint32_t tmem_base;
+  volatile uint32_t abort;
+};
+static_assert(sizeof(V2Bars) <= 256, "control block exceeds its shared-memory slot");
+static_assert(2 * 128 * V2Config::SOFTMAX_REGS + 128 * V2Config::PRODUCER_REGS <=
+                  V2Config::THREADS * V2Config::LAUNCH_REGS,
+              "register split exceeds the registers the block launches with");
+static_assert(V2Config::SOFTMAX_REGS % 8 == 0 && V2Config::PRODUCER_REGS % 8 == 0, "setmaxnreg needs multiples of 8");
+
+// Work-unit geometry shared by every role so that all of them walk the same
+// tile sequence.
+struct UnitGeom {
+  int zq, zkv;         // query (b*H + h) and key/value (b*Hkv + hk) slab
+  int q0;              // first query row of Q0 (Q1 starts at q0 + 128)
+  int last[2];         // last KV tile index Q_k needs, -1 if Q_k is empty
+  int ntiles;          // KV tiles in the stream: last[1] + 1 (or last[0] + 1)
+};
+
+__device__ __forceinline__ UnitGeom unit_geom(const FwdParams& p, int u) {
+  UnitGeom g;
+  const int num_pairs = (p.N + 255) / 256;
+  const int bh = p.B * p.H;
+  // Heaviest first: pair index descending, then (b, h).
+  const int pair = num_pairs - 1 - u / bh;
+  const int zq = u % bh;
+  g.zq = zq;
+  const int b = zq / p.H, h = zq % p.H;
+  g.zkv = b * p.Hkv + h / p.h_per_kv;
+  g.q0 = pair * 256;
+  const int nkv = p.num_kv_tiles;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int qk = g.q0 + 128 * k;
+    if (qk >= p.N) {
+      g.last[k] = -1;
+    } else {
+      g.last[k] = p.causal ? min(nkv - 1, (qk + 127) / 128) : nkv - 1;
+    }
+  }
+  g.ntiles = max(g.last[0], g.last[1]) + 1;
+  return g;
+}
+
+// KV tile at stream position `idx` (forward: idx; reverse: ntiles-1-idx).
+__device__ __forceinline__ int stream_tile(const FwdParams& p, const UnitGeom& g, int idx) {
+  return p.reverse ? (g.ntiles - 1 - idx) : idx;
+}
+
+// Wait with a time limit; also gives up as soon as another role aborted.
+__device__ __forceinline__ bool v2_wait(V2Bars* bars, uint64_t* bar, uint32_t parity, uint32_t* err_word,
+                                        uint32_t code) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t spins = 0;
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((++spins & 63u) == 0u) {
+      if (bars->abort) return false;
+      if (globaltimer_ns() - t0 > 2000000000ull) {
+        atomicOr(err_word, code);
+        bars->abort = 1u;
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait used while draining after an abort: ignores the abort flag.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > 500000000ull) return;
+  }
+}
+
+template <bool COUNT>
+__global__ void __launch_bounds__(V2Config::THREADS, 1)
+    fwd_v2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p, uint32_t* err_word) {
+  using C = V2Config;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  V2Bars* bars = reinterpret_cast<V2Bars*>(base + C::OFF_BAR);
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  const int num_units = p.B * p.H * ((p.N + 255) / 256);
+
+  if (tid == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->q_empty, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&bars->s_full[k], 1);
+      mbar_init(&bars->s_free[k], 128);
+      mbar_init(&bars->p_full[k], 128);
+      mbar_init(&bars->o_done[k], 1);
+      mbar_init(&bars->o_free[k], 128);
+    }
+    mbar_init(&bars->drain, 1);
+    bars->abort = 0u;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp >= 8) {
+    // Each role's code sits inside the branch that set its register budget.
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::PRODUCER_REGS));
+  if (warp == 8) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      uint32_t kv_it = 0, q_it = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        const UnitGeom g = unit_geom(p, u);
+        if (q_it > 0) ok = v2_wait(bars, &bars->q_empty, (q_it - 1) & 1, err_word, kErrTimeoutPipe);
+        if (!ok) break;
+        const uint32_t qbytes = (g.last[1] >= 0) ? 2 * C::TILE_BYTES : C::TILE_BYTES;
+        mbar_arrive_expect_tx(&bars->q_full, qbytes);
+        tma_load_3d(base + C::OFF_Q, &tm_q, &bars->q_full, 0, g.q0, g.zq);
+        if (g.last[1] >= 0) tma_load_3d(base + C::OFF_Q + C::TILE_BYTES, &tm_q, &bars->q_full, 0, g.q0 + 128, g.zq);
+        ++q_it;
+        for (int idx = 0; idx < g.ntiles; ++idx) {
+          const int t = stream_tile(p, g, idx);
+          const int st = kv_it % C::STAGES;
+          if (kv_it >= C::STAGES) {
+            ok = v2_wait(bars, &bars->kv_empty[st], ((kv_it / C::STAGES) - 1) & 1, err_word, kErrTimeoutPipe);
+            if (!ok) break;
+          }
+          mbar_arrive_expect_tx(&bars->k_full[st], C::TILE_BYTES);
+          tma_load_3d(base + C::OFF_K + st * C::TILE_BYTES, &tm_k, &bars->k_full[st], 0, t * 128, g.zkv);
+          mbar_arrive_expect_tx(&bars->v_full[st], C::TILE_BYTES);
+          tma_load_3d(base + C::OFF_V + st * C::TILE_BYTES, &tm_v, &bars->v_full[st], 0, t * 128, g.zkv);
+          ++kv_it;
+        }
+      }
+      if (bars->abort) {
+        // Let the loads already issued land before the CTA's shared memory is
+        // released: the last Q pair and the last STAGES K/V tiles.
+        if (q_it > 0) drain_wait(&bars->q_full, (q_it - 1) & 1);
+        for (uint32_t i = (kv_it > C::STAGES ? kv_it - C::STAGES : 0); i < kv_it; ++i) {
+          drain_wait(&bars->k_full[i % C::STAGES], (i / C::STAGES) & 1);
+          drain_wait(&bars->v_full[i % C::STAGES], (i / C::STAGES) & 1);
+        }
+      }
+    }
+  } else if (warp == 9) {
+    // ------------------------------- MMA issuer -------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_e4m3_f32(128, 128, false, false);
+      constexpr uint32_t idesc_pv = idesc_e4m3_f32(128, 128, false, true);
+      const uint32_t sQ = smem_u32(base + C::OFF_Q);
+      const uint32_t sK = smem_u32(base + C::OFF_K);
+      const uint32_t sV = smem_u32(base + C::OFF_V);
+      const uint32_t sP = smem_u32(base + C::OFF_P);
+      uint32_t kv_it = 0, q_it = 0;
+      uint32_t s_it0 = 0, s_it1 = 0, p_it0 = 0, p_it1 = 0, units0 = 0, units1 = 0;
+      bool ok = true;
+
+      // O_k += P^_k V_t (P^_k from its double buffer, V MN-major), k = 0, 1.
+      auto pv_one = [&](int k, int st, uint32_t& p_it, uint32_t units, bool& first) -> bool {
+        if (!v2_wait(bars, &bars->p_full[k], p_it & 1, err_word, kErrTimeoutPipe)) return false;
+        if (first && units > 0) {
+          if (!v2_wait(bars, &bars->o_free[k], (units - 1) & 1, err_word, kErrTimeoutPipe)) return false;
+        }
+        tc_fence_after();
+        const uint32_t tO = tmem + 256 + 128 * k;
+        const uint32_t pa = sP + (2 * k + (p_it & 1)) * C::TILE_BYTES;
+        const uint32_t va = sV + st * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f8_ss(tO, smem_desc(pa + kk * 32, 16, 1024, 2), smem_desc(va + kk * 32 * 128, 128 * 128, 1024, 2),
+                    idesc_pv, !(first && kk == 0));
+        mma_commit(&bars->o_done[k]);
+        ++p_it;
+        first = false;
+        return true;
+      };
+      // S_k = Q_k K_t^T once softmax k has read its previous S.
+      auto s_one = [&](int k, int st, uint32_t& s_it) -> bool {
+        if (s_it > 0 && !v2_wait(bars, &bars->s_free[k], (s_it - 1) & 1, err_word, kErrTimeoutPipe)) return false;
+        tc_fence_after();
+        const uint32_t tS = tmem + 128 * k;
+        const uint32_t qa = sQ + k * C::TILE_BYTES;
+        const uint32_t ka = sK + st * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_f8_ss(tS, smem_desc(qa + kk * 32, 16, 1024, 2), smem_desc(ka + kk * 32, 16, 1024, 2), idesc_qk, kk > 0);
+        mma_commit(&bars->s_full[k]);
+        ++s_it;
+        return true;
+      };
+
+      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        const UnitGeom g = unit_geom(p, u);
+        ok = v2_wait(bars, &bars->q_full, q_it & 1, err_word, kErrTimeoutQ);
+        if (!ok) break;
+        ++q_it;
+        bool first0 = true, first1 = true;
+        int prev_t = -1, prev_st = 0;
+        uint32_t prev_it = 0;
+        for (int idx = 0; idx <= g.ntiles && ok; ++idx) {
+          if (idx < g.ntiles) {
+            const int t = stream_tile(p, g, idx);
+            const int st = kv_it % C::STAGES;
+            ok = v2_wait(bars, &bars->k_full[st], (kv_it / C::STAGES) & 1, err_word, kErrTimeoutKV);
+            if (ok && t <= g.last[0]) ok = s_one(0, st, s_it0);
+            if (ok && t <= g.last[1]) ok = s_one(1, st, s_it1);
+            if (!ok) break;
+            if (idx == g.ntiles - 1) mma_commit(&bars->q_empty);  // every S of the unit issued
+          }
+          if (prev_t >= 0) {
+            // The P V products of the previous tile, then release its stage.
+            ok = v2_wait(bars, &bars->v_full[prev_st], (prev_it / C::STAGES) & 1, err_word, kErrTimeoutKV);
+            if (ok && prev_t <= g.last[0]) ok = pv_one(0, prev_st, p_it0, units0, first0);
+            if (ok && prev_t <= g.last[1]) ok = pv_one(1, prev_st, p_it1, units1, first1);
+            if (!ok) break;
+            mma_commit(&bars->kv_empty[prev_st]);
+          }
+          if (idx < g.ntiles) {
+            prev_t = stream_tile(p, g, idx);
+            prev_st = kv_it % C::STAGES;
+            prev_it = kv_it;
+            ++kv_it;
+          }
+        }
+        if (g.last[0] >= 0) ++units0;
+        if (g.last[1] >= 0) ++units1;
+      }
+      // Every MMA this thread issued has completed before TMEM is released.
+      mma_commit(&bars->drain);
+      drain_wait(&bars->drain, 0);
+    }
+  }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::SOFTMAX_REGS));
+    // ------------------------------- softmax WGs ------------------------------
+    const int k = warp >> 2;  // which query tile of the pair
+    const int r = tid & 127;  // row within the tile == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + 128 * k + lane_off;
+    const uint32_t tO = tmem + 256 + 128 * k + lane_off;
+    const uint32_t sPk = smem_u32(base + C::OFF_P + 2 * k * C::TILE_BYTES);
+    uint32_t s_it = 0, o_it = 0, p_cnt = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+      const UnitGeom g = unit_geom(p, u);
+      const int last = k ? g.last[1] : g.last[0];  // no dynamic indexing: keeps g in registers
+      if (last < 0) continue;
+      const int qk = g.q0 + 128 * k;
+      const int row = qk + r;
+      float m = -INFINITY;  // running max of raw logits
+      float l = 0.0f;
+      uint32_t nzero = 0;
+      int j = 0;
+      for (int idx = 0; idx < g.ntiles; ++idx) {
+        const int t = stream_tile(p, g, idx);
+        if (t > last) continue;
+        const int j0 = t * 128;
+        ok = __all_sync(0xffffffffu, v2_wait(bars, &bars->s_full[k], s_it & 1, err_word, kErrTimeoutMMA));
+        if (!ok) break;  // warp-uniform, so the collective TMEM loads below stay converged
+        ++s_it;
+        tc_fence_after();
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(tS + c * 32, rr);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(rr[i]);
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars->s_free[k]);  // the S buffer may now be overwritten
+
+        const bool edge = (j0 + 128 > p.N) || (p.causal && j0 + 127 > qk);
+        if (edge) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            const int jj = j0 + c;
+            if (jj >= p.N || (p.causal && jj > row)) s[c] = -INFINITY;
+          }
+        }
+        float mt = s[0];
+#pragma unroll
+        for (int c = 1; c < 128; ++c) mt = fmaxf(mt, s[c]);
+        const float m_new = fmaxf(m, mt);
+        const float ms = (m_new == -INFINITY) ? 0.0f : m_new * p.scale_log2;
+        const float alpha = ex2_approx(fmaf(m, p.scale_log2, -ms));
+        float rowsum = 0.0f;
+        // P = 2^(x - m_new); l from FP32 P; P^ = E4M3(P * S) straight to the
+        // P buffer this tile uses (its previous reader, the P V product two
+        // tiles back, is known to be complete).
+        const uint32_t sPb = sPk + (p_cnt & 1) * C::TILE_BYTES;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = ex2_approx(fmaf(s[c], p.scale_log2, -ms));
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) rowsum += s[c] + s[c + 1];
+#pragma unroll
+        for (int c = 0; c < 128; c += 16) {
+          uint32_t w[4];
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            const int cc = c + 4 * q4;
+            w[q4] = cvt_e4m3x2(s[cc] * p.p_scale, s[cc + 1] * p.p_scale) |
+                    (cvt_e4m3x2(s[cc + 2] * p.p_scale, s[cc + 3] * p.p_scale) << 16);
+            if constexpr (COUNT) {
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int jj = j0 + cc + e;
+                const bool visible = row < p.N && jj < p.N && jj >= p.n_sink && (!p.causal || jj <= row);
+                nzero += (visible && ((w[q4] >> (8 * e)) & 0xFFu) == 0u) ? 1u : 0u;
+              }
+            }
+          }
+          const uint32_t off = swizzled_chunk(r, c / 16, 128);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sPb + off), "r"(w[0]), "r"(w[1]), "r"(w[2]),
+                       "r"(w[3])
+                       : "memory");
+        }
+        l = l * alpha + rowsum;
+        m = m_new;
+
+        if (j > 0) {
+          // O_k holds the previous P V only once that product has completed.
+          ok = __all_sync(0xffffffffu, v2_wait(bars, &bars->o_done[k], o_it & 1, err_word, kErrTimeoutMMA));
+          if (!ok) break;
+          ++o_it;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              uint32_t rr[32];
+              tmem_ld32(tO + c * 32, rr);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
+              tmem_st32(tO + c * 32, rr);
+            }
+            tmem_wait_st();
+          }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(&bars->p_full[k]);
+        ++p_cnt;
+        ++j;
+      }
+      if (!ok) break;
+      // Epilogue: the last P V of the unit, then O / (S * l).
+      ok = __all_sync(0xffffffffu, v2_wait(bars, &bars->o_done[k], o_it & 1, err_word, kErrTimeoutMMA));
+      if (!ok) break;
+      ++o_it;
+      tc_fence_after();
+      if constexpr (COUNT) {
+        const uint32_t total = __reduce_add_sync(0xffffffffu, nzero);
+        if (lane == 0 && total) atomicAdd(p.counts + g.zq, static_cast<unsigned long long>(total));
+      } else {
+        const float inv = __frcp_rn(p.p_scale * l);
+        uint8_t* orow = static_cast<uint8_t*>(p.o) + ((static_cast<int64_t>(g.zq) * p.N + row) * 128) * 2;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(tO + c * 32, rr);
+          tmem_wait_ld();
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            w[i] = pack_bf16x2(__uint_as_float(rr[2 * i]) * inv, __uint_as_float(rr[2 * i + 1]) * inv);
+          if (row < p.N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
+        }
+        if (p.lse != nullptr && row < p.N)
+          p.lse[static_cast<int64_t>(g.zq) * p.N + row] = (m * p.scale_log2 + log2f(l)) * 0.6931471805599453f;
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->o_free[k]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fp8attn

@@ -1,0 +1,175 @@
+"""Python binding of libfp8attn (argument marshalling only).
+
+Every step of the attention forward pass runs in the CUDA library; this module
+turns torch tensors into pointers, sizes and a stream, calls the C ABI, and
+turns status codes into exceptions.  PyTorch supplies device memory, streams
+and (for host inputs) the host<->device copies.
+
+Layouts (see include/fp8attn.h): q [B,H,N,d], k and v [B,Hkv,N,d] as E4M3
+(torch.float8_e4m3fn or uint8 bytes), o [B,H,N,d] bfloat16, lse [B,H,N]
+float32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfp8attn.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(5)
+FORWARD, REVERSE = 0, 1
+
+_lock = threading.Lock()
+_lib = None
+
+
+class Fp8AttnError(RuntimeError):
+    """A libfp8attn call returned a non-OK status."""
+
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_str(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m softmax_cast_precision_b200.build` "
+                "(there is no fallback implementation)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.fp8attn_fwd.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, P]
+        L.fp8attn_fwd.restype = i32
+        L.fp8attn_pzero_count.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, P]
+        L.fp8attn_pzero_count.restype = i32
+        L.fp8attn_kv_tile.argtypes = [i32]
+        L.fp8attn_kv_tile.restype = i32
+        L.fp8attn_status_str.argtypes = [i32]
+        L.fp8attn_status_str.restype = ctypes.c_char_p
+        L.fp8attn_check_error.argtypes = [P]
+        L.fp8attn_check_error.restype = i32
+        L.fp8attn_version.restype = i32
+        _lib = L
+        return L
+
+
+def status_str(status: int) -> str:
+    return lib().fp8attn_status_str(int(status)).decode()
+
+
+def kv_tile(d: int) -> int:
+    """Keys per KV block for head dimension d (0 if unsupported)."""
+    return int(lib().fp8attn_kv_tile(int(d)))
+
+
+def _order(kv_order) -> int:
+    if kv_order in (0, "forward", "fwd"):
+        return FORWARD
+    if kv_order in (1, "reverse", "rev"):
+        return REVERSE
+    raise ValueError(f"kv_order must be 'forward'/0 or 'reverse'/1, got {kv_order!r}")
+
+
+def _bytes(t: torch.Tensor) -> torch.Tensor:
+    if t.dtype == torch.float8_e4m3fn:
+        t = t.view(torch.uint8)
+    if t.dtype != torch.uint8:
+        raise TypeError("q, k, v must be torch.float8_e4m3fn or uint8 (E4M3 bytes)")
+    return t.contiguous()
+
+
+def _shapes(q, k, v):
+    if q.dim() != 4 or k.dim() != 4 or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("q must be [B,H,N,d]; k and v [B,Hkv,N,d]")
+    B, H, N, d = q.shape
+    if k.shape[0] != B or k.shape[2] != N or k.shape[3] != d:
+        raise ValueError("q, k, v disagree on B, N or d")
+    return int(B), int(H), int(k.shape[1]), int(N), int(d)
+
+
+def _stream_ptr(device: torch.device, stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr() if t is not None and t.numel() else 0)
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_scale: float = 256.0,
+        kv_order="reverse", with_lse: bool = True, out: torch.Tensor | None = None,
+        lse_out: torch.Tensor | None = None, stream=None, device=None):
+    """Attention forward pass with the static P-cast scale ``p_scale``.
+
+    Device inputs run in place on their device; host inputs are copied to
+    ``device`` (default cuda:0), computed there, and the results copied back
+    to the host.  Returns (o, lse) (lse is None when ``with_lse`` is False).
+    """
+    q, k, v = _bytes(q), _bytes(k), _bytes(v)
+    B, H, Hkv, N, d = _shapes(q, k, v)
+    host = not q.is_cuda
+    if host:
+        dev = torch.device(device if device is not None else "cuda:0")
+        q, k, v = (x.to(dev, non_blocking=True) for x in (q, k, v))
+    dev = q.device
+    if k.device != dev or v.device != dev:
+        raise ValueError("q, k, v must be on the same device")
+    o = out if (out is not None and not host) else torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    lse = None
+    if with_lse:
+        lse = lse_out if (lse_out is not None and not host) else torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    st = lib().fp8attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, N, d, int(bool(causal)),
+                           ctypes.c_float(p_scale), _order(kv_order), _stream_ptr(dev, stream))
+    if st != OK:
+        raise Fp8AttnError(st, "fp8attn_fwd")
+    if host:
+        o_h = out if out is not None else torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        o_h.copy_(o, non_blocking=True)
+        lse_h = None
+        if lse is not None:
+            lse_h = lse_out if lse_out is not None else torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+            lse_h.copy_(lse, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+        return o_h, lse_h
+    return o, lse
+
+
+def pzero_count(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_scale: float = 256.0,
+                kv_order="reverse", n_sink: int = 4, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Per-(b, h) count of visible keys j >= n_sink whose E4M3(P * S) is zero.
+
+    Returns an int64 tensor [B, H] on the inputs' device.
+    """
+    q, k, v = _bytes(q), _bytes(k), _bytes(v)
+    B, H, Hkv, N, d = _shapes(q, k, v)
+    if not q.is_cuda:
+        raise ValueError("pzero_count takes device tensors")
+    counts = out if out is not None else torch.empty((B, H), dtype=torch.int64, device=q.device)
+    st = lib().fp8attn_pzero_count(_ptr(q), _ptr(k), _ptr(v), _ptr(counts), B, H, Hkv, N, d, int(bool(causal)),
+                                   ctypes.c_float(p_scale), _order(kv_order), int(n_sink),
+                                   _stream_ptr(q.device, stream))
+    if st != OK:
+        raise Fp8AttnError(st, "fp8attn_pzero_count")
+    return counts
+
+
+def check_error(stream=None, device=None) -> None:
+    """Synchronise and raise if a device-side bounded wait ran out."""
+    dev = torch.device(device if device is not None else "cuda:0")
+    st = lib().fp8attn_check_error(_stream_ptr(dev, stream))
+    if st != OK:
+        raise Fp8AttnError(st, "fp8attn_check_error")
+
+
+def raw_call(name: str, *args) -> int:
+    """Call a C-ABI entry point with raw arguments (pointers as ints); returns the status."""
+    return int(getattr(lib(), name)(*args))

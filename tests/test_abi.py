@@ -1,0 +1,97 @@
+"""CPU checks of the C-ABI library: it loads without a GPU, exports every
+entry point include/fp8attn.h declares, and rejects invalid arguments before
+touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp8attn.h")
+
+
+@pytest.fixture(scope="module")
+def fp8():
+    from softmax_cast_precision_b200 import build
+
+    build.build()
+    from softmax_cast_precision_b200 import fp8attn
+
+    return fp8attn
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp8attn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ["fp8attn_fwd", "fp8attn_pzero_count", "fp8attn_kv_tile", "fp8attn_status_str",
+                     "fp8attn_check_error"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(fp8):
+    lib = fp8.lib()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", fp8.LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (fp8attn_\w+)", out))
+    assert set(declared_functions()) <= exported
+
+
+def test_library_has_no_oracle_or_torch_dependency(fp8):
+    out = subprocess.run(["ldd", fp8.LIB_PATH], capture_output=True, text=True).stdout
+    assert "oracle" not in out and "torch" not in out and "libcuda.so" not in out
+
+
+def test_host_only_queries(fp8):
+    assert fp8.kv_tile(128) == 128
+    assert fp8.kv_tile(64) == 64
+    assert fp8.kv_tile(96) == 0
+    assert fp8.status_str(0) == "ok"
+    assert fp8.status_str(4) == "device wait timed out"
+    assert fp8.status_str(99) == "unknown status"
+    assert fp8.lib().fp8attn_version() >= 100
+
+
+def _call_fwd(fp8, q=16, k=16, v=16, o=16, B=1, H=2, Hkv=1, N=128, d=128, causal=0, S=256.0, order=1):
+    P = ctypes.c_void_p
+    return fp8.lib().fp8attn_fwd(P(q), P(k), P(v), P(o), P(0), B, H, Hkv, N, d, causal, ctypes.c_float(S), order,
+                                 P(0))
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(d=96), 2), (dict(d=0), 2), (dict(H=3, Hkv=2), 1), (dict(Hkv=0), 1), (dict(H=0), 1),
+    (dict(B=-1), 1), (dict(N=-5), 1), (dict(S=0.0), 1), (dict(S=-1.0), 1), (dict(S=float("inf")), 1),
+    (dict(S=float("nan")), 1), (dict(order=2), 1), (dict(q=0), 1), (dict(k=8), 1), (dict(v=4), 1),
+    (dict(o=0), 1), (dict(o=24), 1), (dict(B=70000), 2),
+])
+def test_invalid_arguments_rejected_without_launch(fp8, kw, expected):
+    assert _call_fwd(fp8, **kw) == expected
+
+
+def test_empty_problems_are_noops(fp8):
+    # nothing to compute: valid, nothing launched, no device needed
+    assert _call_fwd(fp8, N=0) == 0
+    assert _call_fwd(fp8, B=0) == 0
+    assert _call_fwd(fp8, N=0, q=0, k=0, v=0, o=0) == 0
+    P = ctypes.c_void_p
+    assert fp8.lib().fp8attn_pzero_count(P(16), P(16), P(16), P(0), 0, 2, 1, 128, 128, 0, ctypes.c_float(256.0), 1,
+                                         4, P(0)) == 0
+    assert fp8.lib().fp8attn_pzero_count(P(16), P(16), P(16), P(16), 1, 2, 1, 128, 128, 0, ctypes.c_float(256.0), 1,
+                                         -1, P(0)) == 1
+
+
+def test_binding_raises_without_fallback(fp8, monkeypatch):
+    import softmax_cast_precision_b200.fp8attn as mod
+
+    monkeypatch.setattr(mod, "_lib", None)
+    monkeypatch.setattr(mod, "LIB_PATH", "/nonexistent/libfp8attn.so")
+    with pytest.raises(RuntimeError, match="no fallback"):
+        mod.lib()
