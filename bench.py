@@ -39,8 +39,8 @@ METRIC = "FP8 attn fwd TFLOP/s (% of FP8 peak) at N=32K,d=128; output MSE vs FP6
 UNIT = "TFLOP/s"
 WORKLOAD_DESC = ("prefill32k: B=1 H=32 N=32768 d=128 causal, E4M3 Q/K/V, Delta=7 sink (k=4), S=256, "
                  "reverse KV order")
-KERNEL_NAME = "fwd_v1_kernel"
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fwd_prefill32k_traffic.json")
+KERNEL_NAME = "fwd_v2_kernel"
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "fwd_v2_prefill32k_traffic.txt")
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_BF16_TFLOPS = 1590.0
 FP8_OVER_BF16 = 2.0  # nominal dense ratio: 4.5 PF FP8 / 2.25 PF BF16
@@ -171,6 +171,26 @@ def cpu_baseline(q, k, v):
                       f"{WORKLOAD.B * WORKLOAD.H} heads ({flops / 1e12:.3f} TFLOP in {dt:.1f} s)"}
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The maximum of a per-rank scalar over all ranks (identity when alone)."""
+    import torch
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(flop_per_rank: float, world: int, ms_per_step_max: float) -> float:
+    """Whole-job TFLOP/s: every rank's work over the slowest rank's step time."""
+    return flop_per_rank * world / (ms_per_step_max * 1e-3) / 1e12
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank runs its own copy of the workload on its own inputs."""
+    return SEED + rank
+
+
 def mse_vs_fp64(qd, kd, vd, o, rows_np):
     """MSE of the output against exact attention computed in FP64 by PyTorch on
     the same decoded E4M3 inputs, over the given query rows of every head."""
@@ -245,7 +265,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
 
     w = WORKLOAD
-    q, k, v, _ = synthetic.workload_inputs(w, seed=SEED + rank)
+    q, k, v, _ = synthetic.workload_inputs(w, seed=rank_seed(rank))
     qd, kd, vd = (torch.from_numpy(x).to(device) for x in (q, k, v))
     o = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16, device=device)
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=device)
@@ -276,14 +296,10 @@ def main():
         barrier()
     fp8attn.check_error(stream=stream, device=device)
     per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
-    total_ms = ev[0].elapsed_time(ev[-1])
-    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if dist is not None:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), dist, device)
     ms_per_step = total_ms / args.steps
     flops = w.flops()
-    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    value = aggregate_throughput(flops, world, ms_per_step)
 
     # --- end to end through the public API with host buffers ----------------
     qh, kh, vh = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
@@ -301,11 +317,7 @@ def main():
                     device=device)
     e1.record(stream)
     torch.cuda.synchronize(device)
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-    if dist is not None:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, device)
     h2d = q.nbytes + k.nbytes + v.nbytes
     d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
 
@@ -340,7 +352,7 @@ def main():
                      "frac": achieved / peak_burst, "traffic": traffic,
                      "peak_source": f"{peak_src}: bf16 cuBLAS burst x {FP8_OVER_BF16} (FP8/BF16 nominal)",
                      "frac_of_sustained": achieved / peak_sustained},
-        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": aggregate_throughput(flops, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         "clocks": clk.summary(),
         "mse_vs_fp64": {"value": mse, "rows": "256 evenly spaced query rows of each head",

@@ -103,8 +103,16 @@ int launch_v2(const void* q, const void* k, const void* v, FwdParams p, cudaStre
   p.num_q_tiles = (p.N + 127) / 128;
   p.num_kv_tiles = (p.N + 127) / 128;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
-  const int64_t units = static_cast<int64_t>(p.B) * p.H * ((p.N + 255) / 256);
+  const int num_pairs = (p.N + 255) / 256;
+  const int64_t units = static_cast<int64_t>(p.B) * p.H * num_pairs;
   const int grid = static_cast<int>(units < sms ? units : sms);
+  // Scheduling groups: about two waves of units per group, capped so that the
+  // K and V of the heads a group touches (and of the next group, which
+  // overlaps it) stay well inside L2 (126 MB on B200).
+  const int64_t kv_head_bytes = 2ll * p.N * 128;
+  int gh = (2 * grid + num_pairs - 1) / num_pairs;
+  while (gh > 1 && ((gh + p.h_per_kv - 1) / p.h_per_kv + 1) * kv_head_bytes > (48ll << 20)) --gh;
+  p.group_heads = gh < 1 ? 1 : (gh > p.B * p.H ? p.B * p.H : gh);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p, err_word);
   return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
 }

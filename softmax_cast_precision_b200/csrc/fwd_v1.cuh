@@ -32,6 +32,7 @@ struct FwdParams {
   int n_sink;                   // keys j < n_sink are not counted
   int num_q_tiles;
   int num_kv_tiles;
+  int group_heads;               // persistent kernel: (b, h) slabs per scheduling group
   float p_scale;                // S
   float scale_log2;             // log2(e) / sqrt(D)
 };

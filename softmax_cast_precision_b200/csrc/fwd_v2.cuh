@@ -48,8 +48,8 @@ struct V2Config {
   // thread (65536 / 384 rounded down to a multiple of 8); the producer
   // warpgroup gives registers back and the two softmax warpgroups take them.
   static constexpr int LAUNCH_REGS = 168;
-  static constexpr int SOFTMAX_REGS = 224;
-  static constexpr int PRODUCER_REGS = 56;
+  static constexpr int SOFTMAX_REGS = 216;
+  static constexpr int PRODUCER_REGS = 64;
   static constexpr uint32_t TMEM_COLS = 512;
 };
 
@@ -81,9 +81,16 @@ __device__ __forceinline__ UnitGeom unit_geom(const FwdParams& p, int u) {
   UnitGeom g;
   const int num_pairs = (p.N + 255) / 256;
   const int bh = p.B * p.H;
-  // Heaviest first: pair index descending, then (b, h).
-  const int pair = num_pairs - 1 - u / bh;
-  const int zq = u % bh;
+  // Units come in groups of p.group_heads consecutive (b, h) slabs, so that
+  // the CTAs running at any moment share a few heads' K and V in L2; within a
+  // group the longest (latest) query pairs come first for causal balance.
+  const int per_group = p.group_heads * num_pairs;
+  const int grp = u / per_group;
+  const int idx = u - grp * per_group;
+  const int h0 = grp * p.group_heads;
+  const int gsz = min(p.group_heads, bh - h0);
+  const int pair = num_pairs - 1 - idx / gsz;
+  const int zq = h0 + idx % gsz;
   g.zq = zq;
   const int b = zq / p.H, h = zq % p.H;
   g.zkv = b * p.Hkv + h / p.h_per_kv;
@@ -351,35 +358,63 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
 
         const bool edge = (j0 + 128 > p.N) || (p.causal && j0 + 127 > qk);
         if (edge) {
+          // Keys j0 + c with c >= lim are masked: beyond N, or after this
+          // query row under the causal mask.
+          const int lim = min(p.N, p.causal ? row + 1 : p.N) - j0;
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            const int jj = j0 + c;
-            if (jj >= p.N || (p.causal && jj > row)) s[c] = -INFINITY;
-          }
+          for (int c = 0; c < 128; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
         }
-        float mt = s[0];
+        // Running max over this block and the previous maximum: a tree of
+        // three-input maxima (depth 5 instead of a 128-long dependency chain).
+        float m_new;
+        {
+          float t1[43];
 #pragma unroll
-        for (int c = 1; c < 128; ++c) mt = fmaxf(mt, s[c]);
-        const float m_new = fmaxf(m, mt);
+          for (int i = 0; i < 42; ++i) t1[i] = fmax3(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
+          t1[42] = fmax3(s[126], s[127], m);
+          float t2[15];
+#pragma unroll
+          for (int i = 0; i < 14; ++i) t2[i] = fmax3(t1[3 * i], t1[3 * i + 1], t1[3 * i + 2]);
+          t2[14] = t1[42];
+          float t3[5];
+#pragma unroll
+          for (int i = 0; i < 5; ++i) t3[i] = fmax3(t2[3 * i], t2[3 * i + 1], t2[3 * i + 2]);
+          m_new = fmaxf(fmax3(t3[0], t3[1], t3[2]), fmaxf(t3[3], t3[4]));
+        }
         const float ms = (m_new == -INFINITY) ? 0.0f : m_new * p.scale_log2;
         const float alpha = ex2_approx(fmaf(m, p.scale_log2, -ms));
-        float rowsum = 0.0f;
-        // P = 2^(x - m_new); l from FP32 P; P^ = E4M3(P * S) straight to the
-        // P buffer this tile uses (its previous reader, the P V product two
-        // tiles back, is known to be complete).
+        // P = 2^(x - m_new) with x = s * log2(e) / sqrt(d) (packed pairs);
+        // l from FP32 P (eight independent pair sums); P^ = E4M3(P * S)
+        // straight to the P buffer this tile uses (its previous reader, the
+        // P V product two tiles back, is known to be complete).
         const uint32_t sPb = sPk + (p_cnt & 1) * C::TILE_BYTES;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = ex2_approx(fmaf(s[c], p.scale_log2, -ms));
-#pragma unroll
-        for (int c = 0; c < 128; c += 2) rowsum += s[c] + s[c + 1];
+        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t nm2 = f2_pack(-ms, -ms);
+        const uint64_t S2 = f2_pack(p.p_scale, p.p_scale);
+        uint64_t acc[8];
 #pragma unroll
         for (int c = 0; c < 128; c += 16) {
           uint32_t w[4];
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             const int cc = c + 4 * q4;
-            w[q4] = cvt_e4m3x2(s[cc] * p.p_scale, s[cc + 1] * p.p_scale) |
-                    (cvt_e4m3x2(s[cc + 2] * p.p_scale, s[cc + 3] * p.p_scale) << 16);
+            float x0, x1, x2, x3;
+            f2_unpack(f2_fma(f2_pack(s[cc], s[cc + 1]), sc2, nm2), x0, x1);
+            f2_unpack(f2_fma(f2_pack(s[cc + 2], s[cc + 3]), sc2, nm2), x2, x3);
+            const uint64_t pa = f2_pack(ex2_approx(x0), ex2_approx(x1));
+            const uint64_t pb = f2_pack(ex2_approx(x2), ex2_approx(x3));
+            const int ai = (cc / 4) & 3;
+            if (c == 0) {
+              acc[2 * ai] = pa;
+              acc[2 * ai + 1] = pb;
+            } else {
+              acc[2 * ai] = f2_add(acc[2 * ai], pa);
+              acc[2 * ai + 1] = f2_add(acc[2 * ai + 1], pb);
+            }
+            float y0, y1, y2, y3;
+            f2_unpack(f2_mul(pa, S2), y0, y1);
+            f2_unpack(f2_mul(pb, S2), y2, y3);
+            w[q4] = cvt_e4m3x2(y0, y1) | (cvt_e4m3x2(y2, y3) << 16);
             if constexpr (COUNT) {
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
@@ -394,6 +429,14 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
                        "r"(w[3])
                        : "memory");
         }
+        float rowsum;
+        {
+          const uint64_t a01 = f2_add(acc[0], acc[1]), a23 = f2_add(acc[2], acc[3]);
+          const uint64_t a45 = f2_add(acc[4], acc[5]), a67 = f2_add(acc[6], acc[7]);
+          float lo, hi;
+          f2_unpack(f2_add(f2_add(a01, a23), f2_add(a45, a67)), lo, hi);
+          rowsum = lo + hi;
+        }
         l = l * alpha + rowsum;
         m = m_new;
 
@@ -404,15 +447,21 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
           ++o_it;
           tc_fence_after();
           if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+            // O_k *= alpha: four loads, one wait, packed multiplies, four stores.
+            uint32_t o[128];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              uint32_t rr[32];
-              tmem_ld32(tO + c * 32, rr);
-              tmem_wait_ld();
+            for (int c = 0; c < 4; ++c) tmem_ld32(tO + c * 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32 * c));
+            tmem_wait_ld();
+            const uint64_t a2 = f2_pack(alpha, alpha);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) rr[i] = __float_as_uint(__uint_as_float(rr[i]) * alpha);
-              tmem_st32(tO + c * 32, rr);
+            for (int i = 0; i < 128; i += 2) {
+              float lo, hi;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(o[i]), __uint_as_float(o[i + 1])), a2), lo, hi);
+              o[i] = __float_as_uint(lo);
+              o[i + 1] = __float_as_uint(hi);
             }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_st32(tO + c * 32, *reinterpret_cast<uint32_t(*)[32]>(o + 32 * c));
             tmem_wait_st();
           }
         }
