@@ -5,9 +5,9 @@
 //   warps 0-3  softmax for Q0  (TMEM lanes 0..127 of S0 and O0)
 //   warps 4-7  softmax for Q1  (TMEM lanes 0..127 of S1 and O1)
 //   warp  8    TMA producer: Q pair per unit, K and V tiles through a ring
-//   warp  9    MMA issuer: S_k = Q_k K^T and O_k += P^_k V (tcgen05, FP8 E4M3),
-//              and owner of the tensor-memory allocation
-//   warps 10-11 idle (they complete the producer warpgroup for setmaxnreg)
+//   warps 9-10 MMA issuers for Q0 and Q1: S_k = Q_k K^T and O_k += P^_k V
+//              (tcgen05, FP8 E4M3); warp 9 owns the tensor-memory allocation
+//   warp  11   idle (it completes the producer warpgroup for setmaxnreg)
 // Tensor memory: S0 cols [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 // The two softmax warpgroups alternate on the tensor core: while one turns
 // its S tile into P^, the MMA warp runs the other's products, so the tensor
@@ -25,6 +25,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <type_traits>
 
 #include "fwd_v1.cuh"
 #include "sm100_ptx.cuh"
@@ -35,7 +36,7 @@ struct V2Config {
   static constexpr int D = 128;
   static constexpr int BM = 128;
   static constexpr int BN = 128;
-  static constexpr int STAGES = 3;
+  static constexpr int STAGES = 4;              // K ring and V ring depth
   static constexpr int TILE_BYTES = 128 * 128;  // one 128 x 128 E4M3 tile
   static constexpr int OFF_Q = 0;                               // Q0, Q1
   static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;          // K ring
@@ -48,20 +49,25 @@ struct V2Config {
   // thread (65536 / 384 rounded down to a multiple of 8); the producer
   // warpgroup gives registers back and the two softmax warpgroups take them.
   static constexpr int LAUNCH_REGS = 168;
-  static constexpr int SOFTMAX_REGS = 216;
-  static constexpr int PRODUCER_REGS = 64;
+  static constexpr int SOFTMAX_REGS = 208;
+  static constexpr int PRODUCER_REGS = 80;
   static constexpr uint32_t TMEM_COLS = 512;
 };
 
 // Shared-memory control block.
 struct V2Bars {
-  uint64_t q_full, q_empty;
-  uint64_t k_full[V2Config::STAGES], v_full[V2Config::STAGES], kv_empty[V2Config::STAGES];
+  uint64_t q_full[2], q_free;  // q_full[k]: Q_k landed (only for units where Q_k is used)
+  uint64_t k_full[V2Config::STAGES], v_full[V2Config::STAGES];
+  // Ring stages and the Q pair are released by the softmax threads (256
+  // arrivals: each thread arrives twice when the other query tile does not
+  // use the tile), not by tensor-core commits, which stall the MMA pipe.
+  uint64_t k_free[V2Config::STAGES], v_free[V2Config::STAGES];
   uint64_t s_full[2], s_free[2], p_full[2], o_done[2], o_free[2];
-  uint64_t drain;  // MMA warp: all issued tensor-core work complete
+  uint64_t drain[2];  // MMA warps: all issued tensor-core work complete
   uint32_t tmem_base;
   volatile uint32_t abort;
 };
+static_assert(V2Config::SMEM_BYTES <= 232448, "exceeds the 227 KB shared-memory limit per block");
 static_assert(sizeof(V2Bars) <= 256, "control block exceeds its shared-memory slot");
 static_assert(2 * 128 * V2Config::SOFTMAX_REGS + 128 * V2Config::PRODUCER_REGS <=
                   V2Config::THREADS * V2Config::LAUNCH_REGS,
@@ -115,20 +121,20 @@ __device__ __forceinline__ int stream_tile(const FwdParams& p, const UnitGeom& g
 }
 
 // Wait with a time limit; also gives up as soon as another role aborted.
+// Between checks the thread sleeps inside try_wait (suspend hint), so a
+// waiting warp takes no issue slots from the warps sharing its scheduler and
+// still wakes as soon as the phase completes.
 __device__ __forceinline__ bool v2_wait(V2Bars* bars, uint64_t* bar, uint32_t parity, uint32_t* err_word,
                                         uint32_t code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  uint32_t spins = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((++spins & 63u) == 0u) {
-      if (bars->abort) return false;
-      if (globaltimer_ns() - t0 > 2000000000ull) {
-        atomicOr(err_word, code);
-        bars->abort = 1u;
-        return false;
-      }
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
+    if (bars->abort) return false;
+    if (globaltimer_ns() - t0 > 2000000000ull) {
+      atomicOr(err_word, code);
+      bars->abort = 1u;
+      return false;
     }
   }
 }
@@ -140,6 +146,9 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     if (globaltimer_ns() - t0 > 500000000ull) return;
   }
 }
+
+// Pairs out of every eight (16 keys) whose exponentials use the polynomial.
+constexpr int kPolyPairs = 2;
 
 template <bool COUNT>
 __global__ void __launch_bounds__(V2Config::THREADS, 1)
@@ -154,14 +163,25 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
   const int lane = tid & 31;
 
   const int num_units = p.B * p.H * ((p.N + 255) / 256);
+  // Zigzag assignment over the heaviest-first unit list: round r gives CTA c
+  // unit r*G + c on even rounds and r*G + (G-1-c) on odd rounds, so the CTAs
+  // that draw the heavier unit of one round draw the lighter one of the next.
+  // The last round may leave a CTA without a unit (index past the end).
+  auto first_unit = [&](int r) {
+    const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+    const int64_t u = static_cast<int64_t>(r) * G + ((r & 1) ? (G - 1 - c) : c);
+    return u < num_units ? static_cast<int>(u) : num_units;
+  };
 
   if (tid == 0) {
-    mbar_init(&bars->q_full, 1);
-    mbar_init(&bars->q_empty, 1);
+    mbar_init(&bars->q_full[0], 1);
+    mbar_init(&bars->q_full[1], 1);
+    mbar_init(&bars->q_free, 256);
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
-      mbar_init(&bars->kv_empty[s], 1);
+      mbar_init(&bars->k_free[s], 256);
+      mbar_init(&bars->v_free[s], 256);
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(&bars->s_full[k], 1);
@@ -170,7 +190,8 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
       mbar_init(&bars->o_done[k], 1);
       mbar_init(&bars->o_free[k], 128);
     }
-    mbar_init(&bars->drain, 1);
+    mbar_init(&bars->drain[0], 1);
+    mbar_init(&bars->drain[1], 1);
     bars->abort = 0u;
     fence_mbar_init();
   }
@@ -192,26 +213,36 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      uint32_t kv_it = 0, q_it = 0;
+      uint32_t kv_it = 0, q_it = 0, q_done[2] = {0, 0};
       bool ok = true;
-      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+      for (int rr = 0, u = first_unit(0); u < num_units && ok; u = first_unit(++rr)) {
         const UnitGeom g = unit_geom(p, u);
-        if (q_it > 0) ok = v2_wait(bars, &bars->q_empty, (q_it - 1) & 1, err_word, kErrTimeoutPipe);
+        if (q_it > 0) ok = v2_wait(bars, &bars->q_free, (q_it - 1) & 1, err_word, kErrTimeoutPipe);
         if (!ok) break;
-        const uint32_t qbytes = (g.last[1] >= 0) ? 2 * C::TILE_BYTES : C::TILE_BYTES;
-        mbar_arrive_expect_tx(&bars->q_full, qbytes);
-        tma_load_3d(base + C::OFF_Q, &tm_q, &bars->q_full, 0, g.q0, g.zq);
-        if (g.last[1] >= 0) tma_load_3d(base + C::OFF_Q + C::TILE_BYTES, &tm_q, &bars->q_full, 0, g.q0 + 128, g.zq);
+        mbar_arrive_expect_tx(&bars->q_full[0], C::TILE_BYTES);
+        tma_load_3d(base + C::OFF_Q, &tm_q, &bars->q_full[0], 0, g.q0, g.zq);
+        ++q_done[0];
+        if (g.last[1] >= 0) {
+          mbar_arrive_expect_tx(&bars->q_full[1], C::TILE_BYTES);
+          tma_load_3d(base + C::OFF_Q + C::TILE_BYTES, &tm_q, &bars->q_full[1], 0, g.q0 + 128, g.zq);
+          ++q_done[1];
+        }
         ++q_it;
         for (int idx = 0; idx < g.ntiles; ++idx) {
           const int t = stream_tile(p, g, idx);
           const int st = kv_it % C::STAGES;
+          // K is released once both query tiles have read their S for it, V
+          // once both have seen its P V products complete.
           if (kv_it >= C::STAGES) {
-            ok = v2_wait(bars, &bars->kv_empty[st], ((kv_it / C::STAGES) - 1) & 1, err_word, kErrTimeoutPipe);
+            ok = v2_wait(bars, &bars->k_free[st], ((kv_it / C::STAGES) - 1) & 1, err_word, kErrTimeoutPipe);
             if (!ok) break;
           }
           mbar_arrive_expect_tx(&bars->k_full[st], C::TILE_BYTES);
           tma_load_3d(base + C::OFF_K + st * C::TILE_BYTES, &tm_k, &bars->k_full[st], 0, t * 128, g.zkv);
+          if (kv_it >= C::STAGES) {
+            ok = v2_wait(bars, &bars->v_free[st], ((kv_it / C::STAGES) - 1) & 1, err_word, kErrTimeoutPipe);
+            if (!ok) break;
+          }
           mbar_arrive_expect_tx(&bars->v_full[st], C::TILE_BYTES);
           tma_load_3d(base + C::OFF_V + st * C::TILE_BYTES, &tm_v, &bars->v_full[st], 0, t * 128, g.zkv);
           ++kv_it;
@@ -220,99 +251,108 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
       if (bars->abort) {
         // Let the loads already issued land before the CTA's shared memory is
         // released: the last Q pair and the last STAGES K/V tiles.
-        if (q_it > 0) drain_wait(&bars->q_full, (q_it - 1) & 1);
+        if (q_done[0] > 0) drain_wait(&bars->q_full[0], (q_done[0] - 1) & 1);
+        if (q_done[1] > 0) drain_wait(&bars->q_full[1], (q_done[1] - 1) & 1);
         for (uint32_t i = (kv_it > C::STAGES ? kv_it - C::STAGES : 0); i < kv_it; ++i) {
           drain_wait(&bars->k_full[i % C::STAGES], (i / C::STAGES) & 1);
           drain_wait(&bars->v_full[i % C::STAGES], (i / C::STAGES) & 1);
         }
       }
     }
-  } else if (warp == 9) {
-    // ------------------------------- MMA issuer -------------------------------
-    if (lane == 0) {
-      constexpr uint32_t idesc_qk = idesc_e4m3_f32(128, 128, false, false);
-      constexpr uint32_t idesc_pv = idesc_e4m3_f32(128, 128, false, true);
-      const uint32_t sQ = smem_u32(base + C::OFF_Q);
-      const uint32_t sK = smem_u32(base + C::OFF_K);
-      const uint32_t sV = smem_u32(base + C::OFF_V);
-      const uint32_t sP = smem_u32(base + C::OFF_P);
-      uint32_t kv_it = 0, q_it = 0;
-      uint32_t s_it0 = 0, s_it1 = 0, p_it0 = 0, p_it1 = 0, units0 = 0, units1 = 0;
-      bool ok = true;
-
-      // O_k += P^_k V_t (P^_k from its double buffer, V MN-major), k = 0, 1.
-      auto pv_one = [&](int k, int st, uint32_t& p_it, uint32_t units, bool& first) -> bool {
-        if (!v2_wait(bars, &bars->p_full[k], p_it & 1, err_word, kErrTimeoutPipe)) return false;
-        if (first && units > 0) {
-          if (!v2_wait(bars, &bars->o_free[k], (units - 1) & 1, err_word, kErrTimeoutPipe)) return false;
-        }
-        tc_fence_after();
-        const uint32_t tO = tmem + 256 + 128 * k;
-        const uint32_t pa = sP + (2 * k + (p_it & 1)) * C::TILE_BYTES;
-        const uint32_t va = sV + st * C::TILE_BYTES;
+  } else if (warp == 9 || warp == 10) {
+    // ------------------------------- MMA issuers ------------------------------
+    // Warp 9 issues query tile 0's products, warp 10 query tile 1's, each in
+    // a fixed order S_k(i), P V_k(i-1), ... that only depends on its own
+    // softmax warpgroup; both wait with try_wait, which suspends the warp and
+    // takes no issue slots from the softmax warps sharing its scheduler.  The
+    // whole warp runs the loop; lane 0 issues the MMAs and commits (a commit
+    // tracks the MMAs of its own thread).
+    // The role is instantiated once per query tile so that k, and with it
+    // every MMA operand (TMEM addresses and shared-memory descriptors), is a
+    // compile-time constant: with k computed from the warp index at run time
+    // the S products came out wrong on the GPU for every row but the first,
+    // while this form (and an unrolled single-warp form) is exact.
+    auto mma_role = [&](auto kc) {
+    constexpr int k = decltype(kc)::value;
+    constexpr uint32_t idesc_qk = idesc_e4m3_f32(128, 128, false, false);
+    constexpr uint32_t idesc_pv = idesc_e4m3_f32(128, 128, false, true);
+    // Descriptors are built once: a K step of 32 keys/columns moves the
+    // start-address field (bytes >> 4) by 2 for the K-major operands (32
+    // bytes along the row) and by 256 for V (32 rows of 128 bytes).
+    constexpr uint64_t kTile = C::TILE_BYTES >> 4;  // one 16 KB tile in the address field
+    const uint64_t dQ = smem_desc(smem_u32(base + C::OFF_Q), 16, 1024, 2) + k * kTile;
+    const uint64_t dK0 = smem_desc(smem_u32(base + C::OFF_K), 16, 1024, 2);
+    const uint64_t dV0 = smem_desc(smem_u32(base + C::OFF_V), 128 * 128, 1024, 2);
+    const uint64_t dP = smem_desc(smem_u32(base + C::OFF_P), 16, 1024, 2) + 2 * k * kTile;
+    const uint32_t tS = tmem + 128 * k;
+    const uint32_t tO = tmem + 256 + 128 * k;
+    uint32_t kv_base = 0, q_it = 0, s_cnt = 0, p_cnt = 0, units = 0;
+    bool ok = true;
+    auto wait_all = [&](uint64_t* bar, uint32_t parity, uint32_t code) {
+      return __all_sync(0xffffffffu, v2_wait(bars, bar, parity, err_word, code));
+    };
+    for (int rr = 0, u = first_unit(0); u < num_units && ok; u = first_unit(++rr)) {
+      const UnitGeom g = unit_geom(p, u);
+      const uint32_t unit_base = kv_base;
+      kv_base += g.ntiles;
+      const int nk = (k ? g.last[1] : g.last[0]) + 1;  // tiles this query tile needs (0 if empty)
+      if (nk == 0) continue;
+      ok = wait_all(&bars->q_full[k], q_it & 1, kErrTimeoutQ);
+      ++q_it;
+      if (!ok) break;
+      const int lo = p.reverse ? g.ntiles - nk : 0;
+      for (int idx = lo; idx <= lo + nk && ok; ++idx) {
+        if (idx < lo + nk) {
+          // S_k = Q_k K^T once K has landed and softmax k has read its previous S.
+          const uint32_t it = unit_base + idx;
+          const int st = it % C::STAGES;
+          ok = wait_all(&bars->k_full[st], (it / C::STAGES) & 1, kErrTimeoutKV);
+          if (ok && s_cnt > 0) ok = wait_all(&bars->s_free[k], (s_cnt - 1) & 1, kErrTimeoutPipe);
+          if (!ok) break;
+          tc_fence_after();
+          if (lane == 0) {
+            const uint64_t db = dK0 + st * kTile;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f8_ss(tO, smem_desc(pa + kk * 32, 16, 1024, 2), smem_desc(va + kk * 32 * 128, 128 * 128, 1024, 2),
-                    idesc_pv, !(first && kk == 0));
-        mma_commit(&bars->o_done[k]);
-        ++p_it;
-        first = false;
-        return true;
-      };
-      // S_k = Q_k K_t^T once softmax k has read its previous S.
-      auto s_one = [&](int k, int st, uint32_t& s_it) -> bool {
-        if (s_it > 0 && !v2_wait(bars, &bars->s_free[k], (s_it - 1) & 1, err_word, kErrTimeoutPipe)) return false;
-        tc_fence_after();
-        const uint32_t tS = tmem + 128 * k;
-        const uint32_t qa = sQ + k * C::TILE_BYTES;
-        const uint32_t ka = sK + st * C::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_f8_ss(tS, smem_desc(qa + kk * 32, 16, 1024, 2), smem_desc(ka + kk * 32, 16, 1024, 2), idesc_qk, kk > 0);
-        mma_commit(&bars->s_full[k]);
-        ++s_it;
-        return true;
-      };
-
-      for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
-        const UnitGeom g = unit_geom(p, u);
-        ok = v2_wait(bars, &bars->q_full, q_it & 1, err_word, kErrTimeoutQ);
-        if (!ok) break;
-        ++q_it;
-        bool first0 = true, first1 = true;
-        int prev_t = -1, prev_st = 0;
-        uint32_t prev_it = 0;
-        for (int idx = 0; idx <= g.ntiles && ok; ++idx) {
-          if (idx < g.ntiles) {
-            const int t = stream_tile(p, g, idx);
-            const int st = kv_it % C::STAGES;
-            ok = v2_wait(bars, &bars->k_full[st], (kv_it / C::STAGES) & 1, err_word, kErrTimeoutKV);
-            if (ok && t <= g.last[0]) ok = s_one(0, st, s_it0);
-            if (ok && t <= g.last[1]) ok = s_one(1, st, s_it1);
-            if (!ok) break;
-            if (idx == g.ntiles - 1) mma_commit(&bars->q_empty);  // every S of the unit issued
+            for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tS, dQ + 2 * kk, db + 2 * kk, idesc_qk, kk > 0);
+            mma_commit(&bars->s_full[k]);
           }
-          if (prev_t >= 0) {
-            // The P V products of the previous tile, then release its stage.
-            ok = v2_wait(bars, &bars->v_full[prev_st], (prev_it / C::STAGES) & 1, err_word, kErrTimeoutKV);
-            if (ok && prev_t <= g.last[0]) ok = pv_one(0, prev_st, p_it0, units0, first0);
-            if (ok && prev_t <= g.last[1]) ok = pv_one(1, prev_st, p_it1, units1, first1);
-            if (!ok) break;
-            mma_commit(&bars->kv_empty[prev_st]);
-          }
-          if (idx < g.ntiles) {
-            prev_t = stream_tile(p, g, idx);
-            prev_st = kv_it % C::STAGES;
-            prev_it = kv_it;
-            ++kv_it;
-          }
+          __syncwarp();
+          ++s_cnt;
         }
-        if (g.last[0] >= 0) ++units0;
-        if (g.last[1] >= 0) ++units1;
+        if (idx > lo) {
+          // O_k += P^_k V for the previous tile once softmax k has written P^_k
+          // (and, at a unit's first tile, has read out the previous unit's O_k).
+          const uint32_t it = unit_base + idx - 1;
+          const int st = it % C::STAGES;
+          const bool first = (idx - 1 == lo);
+          ok = wait_all(&bars->p_full[k], p_cnt & 1, kErrTimeoutPipe);
+          if (ok) ok = wait_all(&bars->v_full[st], (it / C::STAGES) & 1, kErrTimeoutKV);
+          if (ok && first && units > 0) ok = wait_all(&bars->o_free[k], (units - 1) & 1, kErrTimeoutPipe);
+          if (!ok) break;
+          tc_fence_after();
+          if (lane == 0) {
+            const uint64_t da = dP + (p_cnt & 1) * kTile, db = dV0 + st * kTile;
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tO, da + 2 * kk, db + 256 * kk, idesc_pv, !(first && kk == 0));
+            mma_commit(&bars->o_done[k]);
+          }
+          __syncwarp();
+          ++p_cnt;
+        }
       }
-      // Every MMA this thread issued has completed before TMEM is released.
-      mma_commit(&bars->drain);
-      drain_wait(&bars->drain, 0);
+      ++units;
+    }
+    // Every MMA lane 0 issued has completed before TMEM is released.
+    if (lane == 0) {
+      mma_commit(&bars->drain[k]);
+      drain_wait(&bars->drain[k], 0);
+    }
+    __syncwarp();
+    };
+    if (warp == 9) {
+      mma_role(std::integral_constant<int, 0>{});
+    } else {
+      mma_role(std::integral_constant<int, 1>{});
     }
   }
   } else {
@@ -325,11 +365,17 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
     const uint32_t tO = tmem + 256 + 128 * k + lane_off;
     const uint32_t sPk = smem_u32(base + C::OFF_P + 2 * k * C::TILE_BYTES);
     uint32_t s_it = 0, o_it = 0, p_cnt = 0;
+    uint32_t kv_base = 0;  // stream position of the unit's first KV tile (ring stage bookkeeping)
     bool ok = true;
-    for (int u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+    for (int rr = 0, u = first_unit(0); u < num_units && ok; u = first_unit(++rr)) {
       const UnitGeom g = unit_geom(p, u);
       const int last = k ? g.last[1] : g.last[0];  // no dynamic indexing: keeps g in registers
+      const int last_other = k ? g.last[0] : g.last[1];
+      const uint32_t unit_base = kv_base;
+      kv_base += g.ntiles;
       if (last < 0) continue;
+      int prev_stage = 0;
+      uint32_t prev_cnt = 2;
       const int qk = g.q0 + 128 * k;
       const int row = qk + r;
       float m = -INFINITY;  // running max of raw logits
@@ -345,44 +391,73 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         ++s_it;
         tc_fence_after();
         float s[128];
+        // Two halves: the second load is in flight while the first half's
+        // maximum is formed.
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t rr[32];
           tmem_ld32(tS + c * 32, rr);
 #pragma unroll
           for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(rr[i]);
         }
         tmem_wait_ld();
+#pragma unroll
+        for (int c = 2; c < 4; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(tS + c * 32, rr);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(rr[i]);
+        }
+        // Keys j0 + c with c >= lim are masked: beyond N, or after this query
+        // row under the causal mask (edge blocks only).
+        const bool edge = (j0 + 128 > p.N) || (p.causal && j0 + 127 > qk);
+        const int lim = edge ? min(p.N, p.causal ? row + 1 : p.N) - j0 : 128;
+        if (edge) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+        }
+        float half_max;
+        {
+          float h1[22];
+#pragma unroll
+          for (int i = 0; i < 21; ++i) h1[i] = fmax3(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
+          h1[21] = fmaxf(s[63], m);
+          float h2[8];
+#pragma unroll
+          for (int i = 0; i < 7; ++i) h2[i] = fmax3(h1[3 * i], h1[3 * i + 1], h1[3 * i + 2]);
+          h2[7] = h1[21];
+          half_max = fmaxf(fmax3(fmax3(h2[0], h2[1], h2[2]), fmax3(h2[3], h2[4], h2[5]), h2[6]), h2[7]);
+        }
+        tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&bars->s_free[k]);  // the S buffer may now be overwritten
+        // This S has completed, so the K stage it read (and, at the unit's
+        // last tile, the Q pair) may be refilled once the other query tile is
+        // done with them too; a tile it does not use counts twice here.
+        const int stage = static_cast<int>((unit_base + idx) % C::STAGES);
+        const uint32_t cnt = (t <= last_other) ? 1u : 2u;
+        mbar_arrive_cnt(&bars->k_free[stage], cnt);
+        if (p.reverse ? (t == 0) : (t == last)) mbar_arrive_cnt(&bars->q_free, last_other >= 0 ? 1u : 2u);
 
-        const bool edge = (j0 + 128 > p.N) || (p.causal && j0 + 127 > qk);
         if (edge) {
-          // Keys j0 + c with c >= lim are masked: beyond N, or after this
-          // query row under the causal mask.
-          const int lim = min(p.N, p.causal ? row + 1 : p.N) - j0;
 #pragma unroll
-          for (int c = 0; c < 128; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
+          for (int c = 64; c < 128; ++c) s[c] = (c < lim) ? s[c] : -INFINITY;
         }
-        // Running max over this block and the previous maximum: a tree of
-        // three-input maxima (depth 5 instead of a 128-long dependency chain).
+        // Running max over this block and the previous maximum: trees of
+        // three-input maxima (short dependency chains).
         float m_new;
         {
-          float t1[43];
+          float t1[22];
 #pragma unroll
-          for (int i = 0; i < 42; ++i) t1[i] = fmax3(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
-          t1[42] = fmax3(s[126], s[127], m);
-          float t2[15];
+          for (int i = 0; i < 21; ++i) t1[i] = fmax3(s[64 + 3 * i], s[65 + 3 * i], s[66 + 3 * i]);
+          t1[21] = fmaxf(s[127], half_max);
+          float t2[8];
 #pragma unroll
-          for (int i = 0; i < 14; ++i) t2[i] = fmax3(t1[3 * i], t1[3 * i + 1], t1[3 * i + 2]);
-          t2[14] = t1[42];
-          float t3[5];
-#pragma unroll
-          for (int i = 0; i < 5; ++i) t3[i] = fmax3(t2[3 * i], t2[3 * i + 1], t2[3 * i + 2]);
-          m_new = fmaxf(fmax3(t3[0], t3[1], t3[2]), fmaxf(t3[3], t3[4]));
+          for (int i = 0; i < 7; ++i) t2[i] = fmax3(t1[3 * i], t1[3 * i + 1], t1[3 * i + 2]);
+          t2[7] = t1[21];
+          m_new = fmaxf(fmax3(fmax3(t2[0], t2[1], t2[2]), fmax3(t2[3], t2[4], t2[5]), t2[6]), t2[7]);
         }
         const float ms = (m_new == -INFINITY) ? 0.0f : m_new * p.scale_log2;
-        const float alpha = ex2_approx(fmaf(m, p.scale_log2, -ms));
         // P = 2^(x - m_new) with x = s * log2(e) / sqrt(d) (packed pairs);
         // l from FP32 P (eight independent pair sums); P^ = E4M3(P * S)
         // straight to the P buffer this tile uses (its previous reader, the
@@ -401,8 +476,11 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
             float x0, x1, x2, x3;
             f2_unpack(f2_fma(f2_pack(s[cc], s[cc + 1]), sc2, nm2), x0, x1);
             f2_unpack(f2_fma(f2_pack(s[cc + 2], s[cc + 3]), sc2, nm2), x2, x3);
-            const uint64_t pa = f2_pack(ex2_approx(x0), ex2_approx(x1));
-            const uint64_t pb = f2_pack(ex2_approx(x2), ex2_approx(x3));
+            // Of every 16 keys, the last kPolyPairs pairs take the FMA-pipe
+            // polynomial, the rest the MUFU exponential.
+            const uint64_t pa = (2 * q4 >= 8 - kPolyPairs) ? exp2_poly2(x0, x1) : f2_pack(ex2_approx(x0), ex2_approx(x1));
+            const uint64_t pb = (2 * q4 + 1 >= 8 - kPolyPairs) ? exp2_poly2(x2, x3)
+                                                                : f2_pack(ex2_approx(x2), ex2_approx(x3));
             const int ai = (cc / 4) & 3;
             if (c == 0) {
               acc[2 * ai] = pa;
@@ -437,6 +515,11 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
           f2_unpack(f2_add(f2_add(a01, a23), f2_add(a45, a67)), lo, hi);
           rowsum = lo + hi;
         }
+        // Rescale factor 2^(m_old - m_new): exactly 1 when the maximum did not
+        // change (the product m * c is then not recomputed), 0 before the
+        // first visible key.  Formed after the exponentials so that this one
+        // MUFU operation never waits behind them.
+        const float alpha = (m_new == m) ? 1.0f : ex2_approx(fmaf(m, p.scale_log2, -ms));
         l = l * alpha + rowsum;
         m = m_new;
 
@@ -445,6 +528,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
           ok = __all_sync(0xffffffffu, v2_wait(bars, &bars->o_done[k], o_it & 1, err_word, kErrTimeoutMMA));
           if (!ok) break;
           ++o_it;
+          mbar_arrive_cnt(&bars->v_free[prev_stage], prev_cnt);  // the previous tile's V has been read
           tc_fence_after();
           if (__any_sync(0xffffffffu, alpha != 1.0f)) {
             // O_k *= alpha: four loads, one wait, packed multiplies, four stores.
@@ -468,6 +552,8 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(&bars->p_full[k]);
+        prev_stage = stage;
+        prev_cnt = cnt;
         ++p_cnt;
         ++j;
       }
@@ -476,6 +562,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
       ok = __all_sync(0xffffffffu, v2_wait(bars, &bars->o_done[k], o_it & 1, err_word, kErrTimeoutMMA));
       if (!ok) break;
       ++o_it;
+      mbar_arrive_cnt(&bars->v_free[prev_stage], prev_cnt);
       tc_fence_after();
       if constexpr (COUNT) {
         const uint32_t total = __reduce_add_sync(0xffffffffu, nzero);

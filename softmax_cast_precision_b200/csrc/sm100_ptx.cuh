@@ -38,6 +38,11 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// Arrive `count` times at once.
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
                "r"(bytes)
@@ -52,6 +57,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
       : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Non-blocking probe: has the phase with the given parity completed?
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// try_wait with a suspend-time hint: the thread sleeps (taking no issue
+// slots) until the phase completes or about `hint_ns` nanoseconds pass.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
@@ -231,6 +263,33 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
+}
+
+// 2^x for a pair of arguments x <= 0 on the FMA pipes, leaving the
+// exponential unit (MUFU) to the other elements.  Range reduction in the
+// style of Cody and Waite: j = round(x) (by adding 1.5 * 2^23, which leaves j
+// in the low mantissa bits), f = x - j in [-1/2, 1/2], 2^f from a degree-5
+// minimax polynomial (coefficients fitted by gen_exp2_poly.py; relative error
+// 2.3e-7 in float32), and 2^j applied by adding j to the exponent field.
+// Arguments below -125 are clamped there (2^-125 is negligible next to the
+// row maximum's 1 and casts to E4M3 zero), which also maps -inf to a finite
+// tiny value.
+__device__ __forceinline__ uint64_t exp2_poly2(float x0, float x1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  const uint64_t x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t t = f2_add(x, f2_pack(kRound, kRound));
+  const uint64_t j = f2_add(t, f2_pack(-kRound, -kRound));
+  const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), x);
+  uint64_t q = f2_fma(f, f2_pack(0x1.5c08e6p-10f, 0x1.5c08e6p-10f), f2_pack(0x1.3d0c52p-7f, 0x1.3d0c52p-7f));
+  q = f2_fma(q, f, f2_pack(0x1.c6b6e4p-5f, 0x1.c6b6e4p-5f));
+  q = f2_fma(q, f, f2_pack(0x1.ebf918p-3f, 0x1.ebf918p-3f));
+  q = f2_fma(q, f, f2_pack(0x1.62e428p-1f, 0x1.62e428p-1f));
+  q = f2_fma(q, f, f2_pack(0x1.000002p+0f, 0x1.000002p+0f));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
