@@ -15,8 +15,13 @@
  *
  * Conventions shared by every call:
  *   - All tensor arguments are DEVICE pointers to caller-owned memory; the
- *     library keeps no pointer after a call returns and allocates no device
- *     memory.  Pointers must be 16-byte aligned.
+ *     library keeps no pointer after a call returns.  Pointers must be
+ *     16-byte aligned.  For d = 128 each call takes a 256-byte work-unit
+ *     counter from a per-device stream-ordered memory pool the library
+ *     creates on first use (cudaMallocFromPoolAsync on the call's stream,
+ *     returned with cudaFreeAsync on the same stream before the call
+ *     returns; the pool keeps its memory mapped for reuse), so concurrent
+ *     calls on different streams are independent.
  *   - Layouts are contiguous, row-major, with the head dimension innermost:
  *       q    [B, H,   N, d]  E4M3 bytes (OCP E4M3FN)
  *       k, v [B, Hkv, N, d]  E4M3 bytes

@@ -1,6 +1,8 @@
 // api.cu -- the C ABI of libfp8attn (declared in include/fp8attn.h): argument
-// validation, TMA tensor-map construction and kernel launch.  No allocation:
-// every tensor is caller-owned device memory.
+// validation, TMA tensor-map construction and kernel launch.  Every tensor is
+// caller-owned device memory; the only device memory the library touches
+// besides it is a per-call 256-byte scheduler block from the stream-ordered
+// allocator (d = 128) and a module-static error word.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -72,6 +74,32 @@ int validate(const void* q, const void* k, const void* v, int B, int H, int Hkv,
   return FP8ATTN_OK;
 }
 
+// Per-device stream-ordered pool for the per-call scheduler counter.  Its
+// release threshold is unbounded, so blocks freed back to it stay mapped and
+// later allocations cost no device-side work (the device's default pool
+// unmaps freed memory at every synchronisation, which made calls slow and
+// erratic).
+cudaMemPool_t sched_pool() {
+  static std::mutex mu;
+  static cudaMemPool_t pools[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!pools[dev]) {
+    cudaMemPoolProps props;
+    std::memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return nullptr;
+    uint64_t threshold = ~0ull;
+    if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &threshold) != cudaSuccess) return nullptr;
+    pools[dev] = pool;
+  }
+  return pools[dev];
+}
+
 int num_sms() {
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -113,8 +141,22 @@ int launch_v2(const void* q, const void* k, const void* v, FwdParams p, cudaStre
   int gh = (2 * grid + num_pairs - 1) / num_pairs;
   while (gh > 1 && ((gh + p.h_per_kv - 1) / p.h_per_kv + 1) * kv_head_bytes > (48ll << 20)) --gh;
   p.group_heads = gh < 1 ? 1 : (gh > p.B * p.H ? p.B * p.H : gh);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p, err_word);
-  return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
+  // Work units are claimed from a counter that must be zero at launch; it
+  // lives in a 256-byte block from the library's stream-ordered pool for the
+  // duration of this call, so concurrent calls on other streams never share it.
+  void* sched = nullptr;
+  cudaMemPool_t pool = sched_pool();
+  if (!pool || cudaMallocFromPoolAsync(&sched, 256, pool, stream) != cudaSuccess) return FP8ATTN_ERR_CUDA;
+  int status = FP8ATTN_OK;
+  if (cudaMemsetAsync(sched, 0, sizeof(unsigned int), stream) != cudaSuccess) {
+    status = FP8ATTN_ERR_CUDA;
+  } else {
+    p.sched = static_cast<unsigned int*>(sched);
+    kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p, err_word);
+    if (cudaGetLastError() != cudaSuccess) status = FP8ATTN_ERR_CUDA;
+  }
+  if (cudaFreeAsync(sched, stream) != cudaSuccess) status = FP8ATTN_ERR_CUDA;
+  return status;
 }
 
 template <int D, bool COUNT>

@@ -33,6 +33,7 @@ struct FwdParams {
   int num_q_tiles;
   int num_kv_tiles;
   int group_heads;               // persistent kernel: (b, h) slabs per scheduling group
+  unsigned int* sched;           // persistent kernel: work-unit counter, zero at launch
   float p_scale;                // S
   float scale_log2;             // log2(e) / sqrt(D)
 };

@@ -43,7 +43,7 @@ struct V2Config {
   static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;     // V ring
   static constexpr int OFF_P = OFF_V + STAGES * TILE_BYTES;     // P0 x2, P1 x2 (double-buffered)
   static constexpr int OFF_BAR = OFF_P + 4 * TILE_BYTES;
-  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // control block + alignment slack
+  static constexpr int SMEM_BYTES = OFF_BAR + 320 + 1024;  // control block + alignment slack
   static constexpr int THREADS = 384;  // 3 warpgroups
   // Register split (setmaxnreg): the block launches with 168 registers per
   // thread (65536 / 384 rounded down to a multiple of 8); the producer
@@ -64,11 +64,15 @@ struct V2Bars {
   uint64_t k_free[V2Config::STAGES], v_free[V2Config::STAGES];
   uint64_t s_full[2], s_free[2], p_full[2], o_done[2], o_free[2];
   uint64_t drain[2];  // MMA warps: all issued tensor-core work complete
+  // Dynamic schedule: the producer fetches unit ids from a global counter and
+  // hands them to the other roles through a two-slot queue.
+  uint64_t unit_full[2], unit_empty[2];
+  int unit_id[2];
   uint32_t tmem_base;
   volatile uint32_t abort;
 };
 static_assert(V2Config::SMEM_BYTES <= 232448, "exceeds the 227 KB shared-memory limit per block");
-static_assert(sizeof(V2Bars) <= 256, "control block exceeds its shared-memory slot");
+static_assert(sizeof(V2Bars) <= 320, "control block exceeds its shared-memory slot");
 static_assert(2 * 128 * V2Config::SOFTMAX_REGS + 128 * V2Config::PRODUCER_REGS <=
                   V2Config::THREADS * V2Config::LAUNCH_REGS,
               "register split exceeds the registers the block launches with");
@@ -147,6 +151,10 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Readers of each published unit id: lane 0 of the two MMA warps and every
+// thread of the two softmax warpgroups.
+constexpr uint32_t kUnitReaders = 2 + 256;
+
 // Pairs out of every eight (16 keys) whose exponentials use the polynomial.
 constexpr int kPolyPairs = 2;
 
@@ -163,14 +171,16 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
   const int lane = tid & 31;
 
   const int num_units = p.B * p.H * ((p.N + 255) / 256);
-  // Zigzag assignment over the heaviest-first unit list: round r gives CTA c
-  // unit r*G + c on even rounds and r*G + (G-1-c) on odd rounds, so the CTAs
-  // that draw the heavier unit of one round draw the lighter one of the next.
-  // The last round may leave a CTA without a unit (index past the end).
-  auto first_unit = [&](int r) {
-    const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
-    const int64_t u = static_cast<int64_t>(r) * G + ((r & 1) ? (G - 1 - c) : c);
-    return u < num_units ? static_cast<int>(u) : num_units;
+  // Work units are handed out dynamically in the heaviest-first, head-grouped
+  // order of unit_geom: the producer takes the next index from the global
+  // counter p.sched (zero at launch) and passes it to the other roles.
+  // next_unit(it) returns the it-th unit of this CTA (-1 when none is left).
+  auto next_unit = [&](uint32_t it, bool reader_arrives) -> int {
+    const int slot = it & 1;
+    if (!v2_wait(bars, &bars->unit_full[slot], (it >> 1) & 1, err_word, kErrTimeoutPipe)) return -1;
+    const int u = *reinterpret_cast<volatile int*>(&bars->unit_id[slot]);
+    if (reader_arrives) mbar_arrive(&bars->unit_empty[slot]);
+    return u;
   };
 
   if (tid == 0) {
@@ -192,6 +202,10 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
     }
     mbar_init(&bars->drain[0], 1);
     mbar_init(&bars->drain[1], 1);
+    for (int s2 = 0; s2 < 2; ++s2) {
+      mbar_init(&bars->unit_full[s2], 1);
+      mbar_init(&bars->unit_empty[s2], kUnitReaders);
+    }
     bars->abort = 0u;
     fence_mbar_init();
   }
@@ -215,7 +229,17 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
       tma_prefetch_desc(&tm_v);
       uint32_t kv_it = 0, q_it = 0, q_done[2] = {0, 0};
       bool ok = true;
-      for (int rr = 0, u = first_unit(0); u < num_units && ok; u = first_unit(++rr)) {
+      for (uint32_t u_it = 0; ok; ++u_it) {
+        // Claim the next unit and publish it (slot reuse waits until every
+        // reader has taken the unit published two claims ago).
+        const int slot = u_it & 1;
+        if (u_it >= 2 && !v2_wait(bars, &bars->unit_empty[slot], ((u_it >> 1) - 1) & 1, err_word, kErrTimeoutPipe))
+          break;
+        int u = static_cast<int>(atomicAdd(p.sched, 1u));
+        if (u >= num_units) u = -1;
+        bars->unit_id[slot] = u;
+        mbar_arrive(&bars->unit_full[slot]);
+        if (u < 0) break;
         const UnitGeom g = unit_geom(p, u);
         if (q_it > 0) ok = v2_wait(bars, &bars->q_free, (q_it - 1) & 1, err_word, kErrTimeoutPipe);
         if (!ok) break;
@@ -291,7 +315,9 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
     auto wait_all = [&](uint64_t* bar, uint32_t parity, uint32_t code) {
       return __all_sync(0xffffffffu, v2_wait(bars, bar, parity, err_word, code));
     };
-    for (int rr = 0, u = first_unit(0); u < num_units && ok; u = first_unit(++rr)) {
+    for (uint32_t u_it = 0; ok; ++u_it) {
+      const int u = __shfl_sync(0xffffffffu, next_unit(u_it, lane == 0), 0);
+      if (u < 0) break;
       const UnitGeom g = unit_geom(p, u);
       const uint32_t unit_base = kv_base;
       kv_base += g.ntiles;
@@ -367,7 +393,9 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
     uint32_t s_it = 0, o_it = 0, p_cnt = 0;
     uint32_t kv_base = 0;  // stream position of the unit's first KV tile (ring stage bookkeeping)
     bool ok = true;
-    for (int rr = 0, u = first_unit(0); u < num_units && ok; u = first_unit(++rr)) {
+    for (uint32_t u_it = 0; ok; ++u_it) {
+      const int u = __shfl_sync(0xffffffffu, next_unit(u_it, true), 0);
+      if (u < 0) break;
       const UnitGeom g = unit_geom(p, u);
       const int last = k ? g.last[1] : g.last[0];  // no dynamic indexing: keeps g in registers
       const int last_other = k ? g.last[0] : g.last[1];
