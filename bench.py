@@ -15,6 +15,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -58,12 +59,24 @@ def parse_args():
     return ap.parse_args()
 
 
+_CODE_TOKENS = re.compile(r'"(?:\\.|[^"\\])*"|\'(?:\\.|[^\'\\])*\'|//[^\n]*|/\*.*?\*/', re.S)
+
+
+def _strip_comments(src: str) -> str:
+    """C/C++ source without comments and with whitespace collapsed (string literals kept)."""
+    code = _CODE_TOKENS.sub(lambda m: " " if m.group(0)[0] == "/" else m.group(0), src)
+    return " ".join(code.split())
+
+
 def kernel_source_hash() -> str:
+    """Hash of the CUDA sources' code, insensitive to comments and layout."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "softmax_cast_precision_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as fh:
-            h.update(name.encode() + fh.read())
+        if not name.endswith((".cu", ".cuh")):
+            continue
+        with open(os.path.join(csrc, name), encoding="utf-8") as fh:
+            h.update(name.encode() + _strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

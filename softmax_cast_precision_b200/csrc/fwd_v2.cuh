@@ -1,7 +1,8 @@
 // fwd_v2.cuh -- persistent, warp-specialised sm_100a forward kernel (d = 128).
 //
-// One CTA per SM walks a static, heaviest-first list of work units; a unit is
-// a pair of adjacent 128-row query tiles (Q0, Q1) of one (batch, head).  Roles:
+// One CTA per SM claims work units from a global counter, in a head-grouped,
+// heaviest-first order; a unit is a pair of adjacent 128-row query tiles
+// (Q0, Q1) of one (batch, head).  Roles:
 //   warps 0-3  softmax for Q0  (TMEM lanes 0..127 of S0 and O0)
 //   warps 4-7  softmax for Q1  (TMEM lanes 0..127 of S1 and O1)
 //   warp  8    TMA producer: Q pair per unit, K and V tiles through a ring
@@ -10,8 +11,8 @@
 //   warp  11   idle (it completes the producer warpgroup for setmaxnreg)
 // Tensor memory: S0 cols [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 // The two softmax warpgroups alternate on the tensor core: while one turns
-// its S tile into P^, the MMA warp runs the other's products, so the tensor
-// core and the exponential/convert pipes overlap.
+// its S tile into P^, the other query tile's MMA warp runs its products, so
+// the tensor core and the exponential/convert pipes overlap.
 //
 // Per KV tile and query row the arithmetic is that of the simple kernel:
 // running max over every block, P = 2^(x - m), l from unquantised P, the
