@@ -59,8 +59,15 @@ enum fp8attn_status {
     FP8ATTN_ERR_INVALID_ARG = 1, /* a size, pointer, alignment or scale is invalid */
     FP8ATTN_ERR_UNSUPPORTED = 2, /* valid but not supported here (d, device)       */
     FP8ATTN_ERR_CUDA = 3,        /* a CUDA runtime or driver call failed            */
-    FP8ATTN_ERR_TIMEOUT = 4      /* a device-side bounded wait ran out              */
+    FP8ATTN_ERR_TIMEOUT = 4,     /* a device-side bounded wait ran out              */
+    FP8ATTN_ERR_SCRATCH_LIMIT = 5 /* too large for fp8attn_fwd_noalloc's fixed scratch */
 };
+
+/* Size of the device array that fp8attn_fwd_noalloc uses as scratch (one per
+ * device), and the most work units (B * H * ceil(N / 256), d = 128) one of
+ * its calls accepts: its counter is one 32-bit word of that array. */
+#define FP8ATTN_NOALLOC_SCRATCH_BYTES 256
+#define FP8ATTN_NOALLOC_MAX_UNITS 2147418112LL /* 2^31 - 2^16 */
 
 /*
  * Forward pass.  Writes o (bfloat16, O = sum_j P^_j v_j / (S * l)) and, when
@@ -86,6 +93,39 @@ int fp8attn_pzero_count(const void* q, const void* k, const void* v,
                         unsigned long long* counts,
                         int B, int H, int Hkv, int N, int d, int causal,
                         float p_scale, int kv_order, int n_sink, void* stream);
+
+/*
+ * Allocation-free forward pass.  The pages have no counterpart of this call:
+ * it is an interface for callers that cannot let the library allocate device
+ * memory -- programs that hand the whole device memory to their own allocator
+ * up front and budget it exactly, and latency-bound loops in which an
+ * allocation (which may block, grow a pool or fail under fragmentation) at an
+ * unpredictable moment is not acceptable.
+ *
+ * Arguments, layouts, results and status codes are those of fp8attn_fwd, and
+ * so are the outputs on every input both accept.  The differences:
+ *   - Scratch.  For d = 128 the persistent kernel's work-unit counter is word
+ *     0 of one library-static device array of FP8ATTN_NOALLOC_SCRATCH_BYTES
+ *     bytes (one array per device), not a per-call block.  Each call zeroes
+ *     the counter on `stream` (cudaMemsetAsync) before its launch.  No call
+ *     allocates or frees device memory.  d = 64 runs a kernel that needs no
+ *     scratch.
+ *   - Set-up.  The first call on a device (the device current at the call)
+ *     looks up the array's address with cudaGetSymbolAddress, loads both
+ *     forward kernels and sets their shared-memory limits; it returns
+ *     FP8ATTN_ERR_CUDA if any of that fails.  Make that first call before any
+ *     stream capture begins.
+ *   - Sharing.  Every call on a device uses the same array.  Calls that can
+ *     overlap on the device (streams without ordering between them, or
+ *     several host threads) race on the counter and give wrong results:
+ *     order them, e.g. issue them all on one stream.
+ *   - Limit.  A d = 128 problem with more than FP8ATTN_NOALLOC_MAX_UNITS work
+ *     units is rejected with FP8ATTN_ERR_SCRATCH_LIMIT before anything is
+ *     launched.
+ */
+int fp8attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int H, int Hkv, int N, int d, int causal,
+                        float p_scale, int kv_order, void* stream);
 
 /* KV block size B_c the kernels use for head dimension d (0 if d is
  * unsupported).  The query block is always 128 rows. */

@@ -2,7 +2,8 @@
 // validation, TMA tensor-map construction and kernel launch.  Every tensor is
 // caller-owned device memory; the only device memory the library touches
 // besides it is a per-call 256-byte scheduler block from the stream-ordered
-// allocator (d = 128) and a module-static error word.
+// allocator (fp8attn_fwd, d = 128), the module-static scratch array of
+// fp8attn_fwd_noalloc and a module-static error word.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -20,6 +21,10 @@ namespace fp8attn {
 // Device error word set by bounded waits that run out (one per process and
 // device image; read and cleared by fp8attn_check_error).
 __device__ uint32_t g_error_word;
+
+// Scratch of fp8attn_fwd_noalloc: word 0 is the persistent kernel's work-unit
+// counter.  One array per device image, shared by every such call.
+static __device__ __align__(256) unsigned int g_noalloc_scratch[FP8ATTN_NOALLOC_SCRATCH_BYTES / sizeof(unsigned int)];
 
 namespace {
 
@@ -194,6 +199,77 @@ FwdParams base_params(int B, int H, int Hkv, int N, int causal, float p_scale, i
   return p;
 }
 
+// ---- allocation-free entry point (fp8attn_fwd_noalloc) ----
+
+// Per-device state of the allocation-free entry point, filled once by its
+// first call on that device.
+struct NoallocDevice {
+  bool ready;
+  unsigned int* scratch;  // device address of g_noalloc_scratch
+  uint32_t* err_word;     // device address of g_error_word
+  int sms;
+};
+
+int noalloc_setup(NoallocDevice** out) {
+  static std::mutex mu;
+  static NoallocDevice devs[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  NoallocDevice& s = devs[dev];
+  if (!s.ready) {
+    if (!get_encode_fn()) return FP8ATTN_ERR_CUDA;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&s.scratch), g_noalloc_scratch) != cudaSuccess)
+      return FP8ATTN_ERR_CUDA;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&s.err_word), g_error_word) != cudaSuccess)
+      return FP8ATTN_ERR_CUDA;
+    // Load both forward kernels and set their shared-memory limits now, so
+    // that later calls do no module loading.
+    auto k2 = fwd_v2_kernel<false>;
+    auto k1 = fwd_v1_kernel<64, false>;
+    cudaFuncAttributes attr;
+    if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, V2Config::SMEM_BYTES) !=
+            cudaSuccess ||
+        cudaFuncGetAttributes(&attr, k2) != cudaSuccess)
+      return FP8ATTN_ERR_CUDA;
+    if (attr.numRegs != V2Config::LAUNCH_REGS) return FP8ATTN_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, V1Config<64>::SMEM_BYTES) !=
+            cudaSuccess ||
+        cudaFuncGetAttributes(&attr, k1) != cudaSuccess)
+      return FP8ATTN_ERR_CUDA;
+    s.sms = num_sms();
+    if (s.sms <= 0) return FP8ATTN_ERR_CUDA;
+    s.ready = true;
+  }
+  *out = &s;
+  return FP8ATTN_OK;
+}
+
+// The persistent kernel with its work-unit counter in g_noalloc_scratch
+// (zeroed on the stream before the launch) instead of a pool block.
+int launch_v2_noalloc(const void* q, const void* k, const void* v, FwdParams p, cudaStream_t stream,
+                      const NoallocDevice& dev) {
+  using C = V2Config;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, 128, p.N, p.B * p.H, 128) || !make_map(&tk, k, 128, p.N, p.B * p.Hkv, 128) ||
+      !make_map(&tv, v, 128, p.N, p.B * p.Hkv, 128))
+    return FP8ATTN_ERR_CUDA;
+  p.num_q_tiles = (p.N + 127) / 128;
+  p.num_kv_tiles = (p.N + 127) / 128;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
+  const int num_pairs = (p.N + 255) / 256;
+  const int64_t units = static_cast<int64_t>(p.B) * p.H * num_pairs;
+  const int grid = static_cast<int>(units < dev.sms ? units : dev.sms);
+  const int64_t kv_head_bytes = 2ll * p.N * 128;
+  int gh = (2 * grid + num_pairs - 1) / num_pairs;
+  while (gh > 1 && ((gh + p.h_per_kv - 1) / p.h_per_kv + 1) * kv_head_bytes > (48ll << 20)) --gh;
+  p.group_heads = gh < 1 ? 1 : (gh > p.B * p.H ? p.B * p.H : gh);
+  if (cudaMemsetAsync(dev.scratch, 0, sizeof(unsigned int), stream) != cudaSuccess) return FP8ATTN_ERR_CUDA;
+  p.sched = dev.scratch;
+  fwd_v2_kernel<false><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p, dev.err_word);
+  return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
+}
+
 }  // namespace
 }  // namespace fp8attn
 
@@ -230,6 +306,24 @@ extern "C" int fp8attn_pzero_count(const void* q, const void* k, const void* v, 
   return d == 128 ? launch_v2<true>(q, k, v, p, s) : launch<64, true>(q, k, v, p, s);
 }
 
+extern "C" int fp8attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                                   int Hkv, int N, int d, int causal, float p_scale, int kv_order, void* stream) {
+  int st = validate(q, k, v, B, H, Hkv, N, d, p_scale, kv_order);
+  if (st != FP8ATTN_OK) return st;
+  if (static_cast<int64_t>(B) * H * N == 0) return FP8ATTN_OK;
+  if (!o || !aligned16(o) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))) return FP8ATTN_ERR_INVALID_ARG;
+  if (d == 128 && static_cast<int64_t>(B) * H * ((N + 255) / 256) > FP8ATTN_NOALLOC_MAX_UNITS)
+    return FP8ATTN_ERR_SCRATCH_LIMIT;
+  NoallocDevice* dev = nullptr;
+  st = noalloc_setup(&dev);
+  if (st != FP8ATTN_OK) return st;
+  FwdParams p = base_params(B, H, Hkv, N, causal, p_scale, kv_order);
+  p.o = o;
+  p.lse = lse;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 128 ? launch_v2_noalloc(q, k, v, p, s, *dev) : launch<64, false>(q, k, v, p, s);
+}
+
 extern "C" int fp8attn_kv_tile(int d) {
   if (d == 128) return V1Config<128>::BN;
   if (d == 64) return V1Config<64>::BN;
@@ -248,6 +342,8 @@ extern "C" const char* fp8attn_status_str(int status) {
       return "CUDA error";
     case FP8ATTN_ERR_TIMEOUT:
       return "device wait timed out";
+    case FP8ATTN_ERR_SCRATCH_LIMIT:
+      return "problem too large for the allocation-free entry point's fixed scratch";
     default:
       return "unknown status";
   }

@@ -20,7 +20,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfp8attn.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(5)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT, ERR_SCRATCH_LIMIT = range(6)
 FORWARD, REVERSE = 0, 1
 
 _lock = threading.Lock()
@@ -49,6 +49,8 @@ def lib() -> ctypes.CDLL:
         P, i32, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.fp8attn_fwd.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, P]
         L.fp8attn_fwd.restype = i32
+        L.fp8attn_fwd_noalloc.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, P]
+        L.fp8attn_fwd_noalloc.restype = i32
         L.fp8attn_pzero_count.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, P]
         L.fp8attn_pzero_count.restype = i32
         L.fp8attn_kv_tile.argtypes = [i32]
@@ -141,6 +143,38 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_sc
         torch.cuda.current_stream(dev).synchronize()
         return o_h, lse_h
     return o, lse
+
+
+def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
+                lse_out: torch.Tensor | None = None, *, causal: bool, p_scale: float = 256.0,
+                kv_order="reverse", stream=None) -> None:
+    """The allocation-free forward pass (C entry point ``fp8attn_fwd_noalloc``).
+
+    For callers that cannot let the library allocate device memory.  All
+    tensors are the caller's, on one device: ``out`` bf16 [B,H,N,d] and the
+    optional ``lse_out`` float32 [B,H,N], both contiguous, are written in
+    place.  Every call on a device shares one fixed scratch array, so calls
+    must not overlap (keep them on one stream); the first call on a device
+    does a one-time set-up and should come before any stream capture.
+    q, k and v must be contiguous: this wrapper makes no copies.
+    """
+    if not all(t.is_contiguous() for t in (q, k, v)):
+        raise ValueError("fwd_noalloc takes contiguous q, k, v")
+    q, k, v = _bytes(q), _bytes(k), _bytes(v)
+    B, H, Hkv, N, d = _shapes(q, k, v)
+    if not q.is_cuda or k.device != q.device or v.device != q.device:
+        raise ValueError("fwd_noalloc takes device tensors on one device")
+    if (out.device != q.device or out.dtype != torch.bfloat16 or tuple(out.shape) != (B, H, N, d)
+            or not out.is_contiguous()):
+        raise ValueError("out must be a contiguous bfloat16 [B,H,N,d] tensor on the inputs' device")
+    if lse_out is not None and (lse_out.device != q.device or lse_out.dtype != torch.float32
+                                or tuple(lse_out.shape) != (B, H, N) or not lse_out.is_contiguous()):
+        raise ValueError("lse_out must be a contiguous float32 [B,H,N] tensor on the inputs' device")
+    st = lib().fp8attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse_out), B, H, Hkv, N, d,
+                                   int(bool(causal)), ctypes.c_float(p_scale), _order(kv_order),
+                                   _stream_ptr(q.device, stream))
+    if st != OK:
+        raise Fp8AttnError(st, "fp8attn_fwd_noalloc")
 
 
 def pzero_count(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_scale: float = 256.0,

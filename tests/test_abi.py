@@ -30,7 +30,7 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for required in ["fp8attn_fwd", "fp8attn_pzero_count", "fp8attn_kv_tile", "fp8attn_status_str",
+    for required in ["fp8attn_fwd", "fp8attn_fwd_noalloc", "fp8attn_pzero_count", "fp8attn_kv_tile", "fp8attn_status_str",
                      "fp8attn_check_error"]:
         assert required in names
 
@@ -60,10 +60,11 @@ def test_host_only_queries(fp8):
     assert fp8.lib().fp8attn_version() >= 100
 
 
-def _call_fwd(fp8, q=16, k=16, v=16, o=16, B=1, H=2, Hkv=1, N=128, d=128, causal=0, S=256.0, order=1):
+def _call_fwd(fp8, q=16, k=16, v=16, o=16, B=1, H=2, Hkv=1, N=128, d=128, causal=0, S=256.0, order=1,
+              entry="fp8attn_fwd"):
     P = ctypes.c_void_p
-    return fp8.lib().fp8attn_fwd(P(q), P(k), P(v), P(o), P(0), B, H, Hkv, N, d, causal, ctypes.c_float(S), order,
-                                 P(0))
+    return getattr(fp8.lib(), entry)(P(q), P(k), P(v), P(o), P(0), B, H, Hkv, N, d, causal, ctypes.c_float(S),
+                                     order, P(0))
 
 
 @pytest.mark.parametrize("kw,expected", [
@@ -72,8 +73,28 @@ def _call_fwd(fp8, q=16, k=16, v=16, o=16, B=1, H=2, Hkv=1, N=128, d=128, causal
     (dict(S=float("nan")), 1), (dict(order=2), 1), (dict(q=0), 1), (dict(k=8), 1), (dict(v=4), 1),
     (dict(o=0), 1), (dict(o=24), 1), (dict(B=70000), 2),
 ])
-def test_invalid_arguments_rejected_without_launch(fp8, kw, expected):
-    assert _call_fwd(fp8, **kw) == expected
+@pytest.mark.parametrize("entry", ["fp8attn_fwd", "fp8attn_fwd_noalloc"])
+def test_invalid_arguments_rejected_without_launch(fp8, kw, expected, entry):
+    assert _call_fwd(fp8, entry=entry, **kw) == expected
+
+
+def _header_define(name):
+    m = re.search(rf"#define {name} (\d+)", open(HEADER).read())
+    return int(m.group(1))
+
+
+def test_noalloc_limits_and_rejection(fp8):
+    assert _header_define("FP8ATTN_NOALLOC_SCRATCH_BYTES") == 256
+    max_units = _header_define("FP8ATTN_NOALLOC_MAX_UNITS")
+    assert max_units == 2**31 - 2**16  # the 32-bit counter ends at units + grid (< 2^16 CTAs)
+    assert fp8.status_str(fp8.ERR_SCRATCH_LIMIT).startswith("problem too large")
+    # 65535 x 65535 heads of one row: 4.29e9 work units, rejected before any device work.
+    assert _call_fwd(fp8, B=65535, H=65535, Hkv=65535, N=1, entry="fp8attn_fwd_noalloc") == fp8.ERR_SCRATCH_LIMIT
+    # d = 64 runs a kernel without scratch and does not hit this limit (only the size checks
+    # shared with fp8attn_fwd, which reject this shape as unsupported).
+    assert _call_fwd(fp8, B=65535, H=65535, Hkv=65535, N=300, d=64,
+                     entry="fp8attn_fwd_noalloc") == fp8.ERR_UNSUPPORTED
+    assert _call_fwd(fp8, N=0, q=0, k=0, v=0, o=0, entry="fp8attn_fwd_noalloc") == 0
 
 
 def test_empty_problems_are_noops(fp8):
