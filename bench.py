@@ -69,14 +69,22 @@ def _strip_comments(src: str) -> str:
 
 
 def kernel_source_hash() -> str:
-    """Hash of the CUDA sources' code, insensitive to comments and layout."""
+    """Hash of the forward kernel's code and its launch configuration.
+
+    Covers the device headers and the host function that sizes the
+    persistent kernel's launch; insensitive to comments and layout.
+    """
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "softmax_cast_precision_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
-        if not name.endswith((".cu", ".cuh")):
+        if not name.endswith(".cuh"):
             continue
         with open(os.path.join(csrc, name), encoding="utf-8") as fh:
             h.update(name.encode() + _strip_comments(fh.read()).encode())
+    with open(os.path.join(csrc, "api.cu"), encoding="utf-8") as fh:
+        api = fh.read()
+    m = re.search(r"\nint launch_v2\(.*?\n}\n", api, re.S)
+    h.update(_strip_comments(m.group(0) if m else api).encode())
     return h.hexdigest()[:16]
 
 
