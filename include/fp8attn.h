@@ -34,8 +34,9 @@
  *   - causal != 0 applies the square, top-left aligned mask (query i sees keys
  *     0..i); KV blocks entirely above the diagonal are skipped.
  *   - The logit scale is fixed at 1/sqrt(d).
- *   - p_scale is the static scale S (finite, > 0).  Powers of two make the
- *     scaling exact in FP32; S > 448 saturates the largest probabilities.
+ *   - p_scale is the static scale S, 2^-64 <= S <= 2^64 (anything else, NaN
+ *     included, is FP8ATTN_ERR_INVALID_ARG).  S > 448 saturates the largest
+ *     probabilities.
  *   - kv_order: 0 = forward (KV block 0 first), 1 = reverse (last block
  *     first).
  *   - stream is a cudaStream_t passed as void* (NULL = legacy default

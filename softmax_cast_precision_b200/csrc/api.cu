@@ -69,7 +69,8 @@ int validate(const void* q, const void* k, const void* v, int B, int H, int Hkv,
              int kv_order) {
   if (B < 0 || N < 0 || H < 1 || Hkv < 1 || H % Hkv != 0) return FP8ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FP8ATTN_ERR_UNSUPPORTED;
-  if (!(p_scale > 0.0f) || !std::isfinite(p_scale)) return FP8ATTN_ERR_INVALID_ARG;
+  // S in [2^-64, 2^64]: the kernels carry S * l and 2^(x + log2 S) in float32.
+  if (!(p_scale >= 0x1p-64f) || !(p_scale <= 0x1p64f)) return FP8ATTN_ERR_INVALID_ARG;
   if (kv_order != 0 && kv_order != 1) return FP8ATTN_ERR_INVALID_ARG;
   if (B > 65535 || H > 65535) return FP8ATTN_ERR_UNSUPPORTED;  // grid y/z limits
   const int64_t zq = static_cast<int64_t>(B) * H;
@@ -196,6 +197,7 @@ FwdParams base_params(int B, int H, int Hkv, int N, int causal, float p_scale, i
   p.causal = causal ? 1 : 0;
   p.reverse = kv_order;
   p.p_scale = p_scale;
+  p.log2_p_scale = static_cast<float>(std::log2(static_cast<double>(p_scale)));
   return p;
 }
 

@@ -36,6 +36,7 @@ struct FwdParams {
   unsigned int* sched;           // persistent kernel: work-unit counter, zero at launch
   float p_scale;                // S
   float scale_log2;             // log2(e) / sqrt(D)
+  float log2_p_scale;           // log2(S), rounded to float
 };
 
 template <int D>

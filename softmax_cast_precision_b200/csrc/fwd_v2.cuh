@@ -487,14 +487,16 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
           m_new = fmaxf(fmax3(fmax3(t2[0], t2[1], t2[2]), fmax3(t2[3], t2[4], t2[5]), t2[6]), t2[7]);
         }
         const float ms = (m_new == -INFINITY) ? 0.0f : m_new * p.scale_log2;
-        // P = 2^(x - m_new) with x = s * log2(e) / sqrt(d) (packed pairs);
-        // l from FP32 P (eight independent pair sums); P^ = E4M3(P * S)
-        // straight to the P buffer this tile uses (its previous reader, the
-        // P V product two tiles back, is known to be complete).
+        // P * S = 2^(x - m_new + log2 S) with x = s * log2(e) / sqrt(d)
+        // (packed pairs): the scale enters the exponent, so one exponential
+        // gives the scaled probability.  Its row sum, l * S, is kept (eight
+        // independent pair sums) and divided out at the end; P^ = E4M3(P * S)
+        // goes straight to the P buffer this tile uses (its previous reader,
+        // the P V product two tiles back, is known to be complete).
         const uint32_t sPb = sPk + (p_cnt & 1) * C::TILE_BYTES;
         const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
-        const uint64_t nm2 = f2_pack(-ms, -ms);
-        const uint64_t S2 = f2_pack(p.p_scale, p.p_scale);
+        const float bias = p.log2_p_scale - ms;
+        const uint64_t nm2 = f2_pack(bias, bias);
         uint64_t acc[8];
 #pragma unroll
         for (int c = 0; c < 128; c += 16) {
@@ -519,8 +521,8 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
               acc[2 * ai + 1] = f2_add(acc[2 * ai + 1], pb);
             }
             float y0, y1, y2, y3;
-            f2_unpack(f2_mul(pa, S2), y0, y1);
-            f2_unpack(f2_mul(pb, S2), y2, y3);
+            f2_unpack(pa, y0, y1);
+            f2_unpack(pb, y2, y3);
             w[q4] = cvt_e4m3x2(y0, y1) | (cvt_e4m3x2(y2, y3) << 16);
             if constexpr (COUNT) {
 #pragma unroll
@@ -549,7 +551,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         // first visible key.  Formed after the exponentials so that this one
         // MUFU operation never waits behind them.
         const float alpha = (m_new == m) ? 1.0f : ex2_approx(fmaf(m, p.scale_log2, -ms));
-        l = l * alpha + rowsum;
+        l = l * alpha + rowsum;  // l * S
         m = m_new;
 
         if (j > 0) {
@@ -587,7 +589,8 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         ++j;
       }
       if (!ok) break;
-      // Epilogue: the last P V of the unit, then O / (S * l).
+      // Epilogue: the last P V of the unit, then O / (S * l) (l already
+      // carries the factor S).
       ok = __all_sync(0xffffffffu, v2_wait(bars, &bars->o_done[k], o_it & 1, err_word, kErrTimeoutMMA));
       if (!ok) break;
       ++o_it;
@@ -597,7 +600,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         const uint32_t total = __reduce_add_sync(0xffffffffu, nzero);
         if (lane == 0 && total) atomicAdd(p.counts + g.zq, static_cast<unsigned long long>(total));
       } else {
-        const float inv = __frcp_rn(p.p_scale * l);
+        const float inv = __frcp_rn(l);  // l holds l * S
         uint8_t* orow = static_cast<uint8_t*>(p.o) + ((static_cast<int64_t>(g.zq) * p.N + row) * 128) * 2;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
@@ -615,7 +618,8 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
           }
         }
         if (p.lse != nullptr && row < p.N)
-          p.lse[static_cast<int64_t>(g.zq) * p.N + row] = (m * p.scale_log2 + log2f(l)) * 0.6931471805599453f;
+          p.lse[static_cast<int64_t>(g.zq) * p.N + row] =
+              (m * p.scale_log2 + (log2f(l) - p.log2_p_scale)) * 0.6931471805599453f;
       }
       tc_fence_before();
       mbar_arrive(&bars->o_free[k]);

@@ -2,7 +2,7 @@
 
 Method (range reduction in the style of Cody and Waite, then a minimax
 polynomial fitted here): 2^x = 2^j * 2^f with j = round(x) and
-f = x - j in [-1/2, 1/2]; 2^f is approximated by a degree-5 polynomial whose
+f = x - j in [-1/2, 1/2]; 2^f is approximated by a degree-4 polynomial whose
 coefficients minimise the maximum relative error on that interval, found by
 the Remez exchange algorithm in float64 and then rounded to float32.
 
@@ -15,7 +15,7 @@ from __future__ import annotations
 
 import numpy as np
 
-DEGREE = 5
+DEGREE = 4
 LO, HI = -0.5, 0.5
 
 

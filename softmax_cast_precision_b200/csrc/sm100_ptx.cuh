@@ -265,26 +265,25 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair of arguments x <= 0 on the FMA pipes, leaving the
+// 2^x for a pair of arguments x <= 64 on the FMA pipes, leaving the
 // exponential unit (MUFU) to the other elements.  Range reduction in the
 // style of Cody and Waite: j = round(x) (by adding 1.5 * 2^23, which leaves j
-// in the low mantissa bits), f = x - j in [-1/2, 1/2], 2^f from a degree-5
+// in the low mantissa bits), f = x - j in [-1/2, 1/2], 2^f from a degree-4
 // minimax polynomial (coefficients fitted by gen_exp2_poly.py; relative error
-// 2.3e-7 in float32), and 2^j applied by adding j to the exponent field.
+// 2.7e-6 in float32), and 2^j applied by adding j to the exponent field.
 // Arguments below -125 are clamped there (2^-125 is negligible next to the
-// row maximum's 1 and casts to E4M3 zero), which also maps -inf to a finite
-// tiny value.
+// row maximum's 2^log2(S) >= 2^-64 and casts to E4M3 zero), which also maps
+// -inf to a finite tiny value.
 __device__ __forceinline__ uint64_t exp2_poly2(float x0, float x1) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
   const uint64_t x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
   const uint64_t t = f2_add(x, f2_pack(kRound, kRound));
   const uint64_t j = f2_add(t, f2_pack(-kRound, -kRound));
   const uint64_t f = f2_fma(j, f2_pack(-1.0f, -1.0f), x);
-  uint64_t q = f2_fma(f, f2_pack(0x1.5c08e6p-10f, 0x1.5c08e6p-10f), f2_pack(0x1.3d0c52p-7f, 0x1.3d0c52p-7f));
-  q = f2_fma(q, f, f2_pack(0x1.c6b6e4p-5f, 0x1.c6b6e4p-5f));
-  q = f2_fma(q, f, f2_pack(0x1.ebf918p-3f, 0x1.ebf918p-3f));
-  q = f2_fma(q, f, f2_pack(0x1.62e428p-1f, 0x1.62e428p-1f));
-  q = f2_fma(q, f, f2_pack(0x1.000002p+0f, 0x1.000002p+0f));
+  uint64_t q = f2_fma(f, f2_pack(0x1.3997d6p-7f, 0x1.3997d6p-7f), f2_pack(0x1.ca144p-5f, 0x1.ca144p-5f));
+  q = f2_fma(q, f, f2_pack(0x1.ec06dap-3f, 0x1.ec06dap-3f));
+  q = f2_fma(q, f, f2_pack(0x1.62e0dcp-1f, 0x1.62e0dcp-1f));
+  q = f2_fma(q, f, f2_pack(0x1.ffffe8p-1f, 0x1.ffffe8p-1f));
   float q0, q1, t0, t1;
   f2_unpack(q, q0, q1);
   f2_unpack(t, t0, t1);

@@ -70,7 +70,7 @@ def _call_fwd(fp8, q=16, k=16, v=16, o=16, B=1, H=2, Hkv=1, N=128, d=128, causal
 @pytest.mark.parametrize("kw,expected", [
     (dict(d=96), 2), (dict(d=0), 2), (dict(H=3, Hkv=2), 1), (dict(Hkv=0), 1), (dict(H=0), 1),
     (dict(B=-1), 1), (dict(N=-5), 1), (dict(S=0.0), 1), (dict(S=-1.0), 1), (dict(S=float("inf")), 1),
-    (dict(S=float("nan")), 1), (dict(order=2), 1), (dict(q=0), 1), (dict(k=8), 1), (dict(v=4), 1),
+    (dict(S=float("nan")), 1), (dict(S=2.0**65), 1), (dict(S=2.0**-65), 1), (dict(order=2), 1), (dict(q=0), 1), (dict(k=8), 1), (dict(v=4), 1),
     (dict(o=0), 1), (dict(o=24), 1), (dict(B=70000), 2),
 ])
 @pytest.mark.parametrize("entry", ["fp8attn_fwd", "fp8attn_fwd_noalloc"])
