@@ -127,3 +127,42 @@ def workload_inputs(w: Workload, seed: int, delta=None, v_mode: str = "normal"):
     """Inputs for a workload (``delta`` overrides the workload's sink strength)."""
     return make_inputs(w.B, w.H, w.Hkv, w.N, w.d, w.delta if delta is None else delta,
                        seed, n_sink=w.n_sink, v_mode=v_mode)
+
+
+def _to_bf16_values(x: np.ndarray) -> np.ndarray:
+    """float32 values rounded to bfloat16 (PyTorch's conversion, round to nearest even)."""
+    import torch
+
+    return torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).to(torch.bfloat16).float().numpy()
+
+
+def make_wide_inputs(B: int, H: int, Hkv: int, N: int, d: int, delta, seed: int,
+                     n_sink: int = 4, outliers: int = 0, outlier_gain: float = 16.0):
+    """Unquantised inputs for the quantisation path: float32 arrays holding bfloat16 values.
+
+    Same sink construction as ``make_inputs`` (q[..., 0] = sqrt(d), sink keys
+    k[..., 0] = Delta), without the E4M3 cast.  ``outliers`` > 0 multiplies
+    that many fixed channels (1 .. outliers) of q and k by ``outlier_gain``,
+    the kind of outlier channel that makes a direct per-block cast lose
+    precision on every other channel.  Draw order: Delta, q, k, v.
+    """
+    if H % Hkv:
+        raise ValueError("H must be a multiple of Hkv")
+    rng = np.random.Generator(np.random.PCG64(seed))
+    deltas = sink_deltas(B, Hkv, delta, rng)
+    q = rng.standard_normal((B, H, N, d), dtype=np.float32)
+    q[..., 0] = math.sqrt(d)
+    k = rng.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    k[..., 0] = 0.0
+    k[:, :, :n_sink, 0] = deltas[:, :, None]
+    if outliers:
+        q[..., 1:1 + outliers] *= outlier_gain
+        k[..., 1:1 + outliers] *= outlier_gain
+    v = rng.standard_normal((B, Hkv, N, d), dtype=np.float32)
+    return _to_bf16_values(q), _to_bf16_values(k), _to_bf16_values(v), deltas
+
+
+def hadamard_signs(d: int, seed: int) -> np.ndarray:
+    """The random +-1 column signs of the rotation (float32 [d]), from a seeded generator."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return np.where(rng.random(d) < 0.5, -1.0, 1.0).astype(np.float32)
