@@ -18,9 +18,9 @@ Readings taken where the page is silent (each is stated where it is used):
   * R = diag(signs) H_d / sqrt(d), H_d the Sylvester Hadamard matrix, signs a
     given +-1 vector (an input, drawn by the seeded generator in
     ``synthetic``).
-  * A block's descale is the smallest power of two s with max|x| <= 448 s
-    (448 = largest E4M3 value), so x / s is exact and never saturates, and
-    s * E4M3(x / s) is exact in float32.
+  * A block's descale is the smallest power of two s >= 2^-126 with
+    max|x| <= 448 s (448 = largest E4M3 value), so x / s is exact and never
+    saturates, and s * E4M3(x / s) is exact in float32.
   * Q and K are scaled per block of 128 rows of one (batch, head) -- the
     query and key tiles of the forward kernel -- and V per (batch, head),
     because a per-tile V scale could not be divided out of the accumulated
@@ -115,17 +115,18 @@ def unrotate_f32(y, signs) -> np.ndarray:
 
 
 def block_scale(amax) -> np.ndarray:
-    """Smallest power of two s with amax <= 448 s (1 where amax is 0), as float32.
+    """Smallest power of two s >= 2^-126 with amax <= 448 s (1 where amax is 0), as float32.
 
     Exact rule on the binary exponent: with amax = m 2^E, m in [1, 2), and
-    448 = 1.75 2^8, s = 2^(E - 8) when m <= 1.75, else 2^(E - 7).
+    448 = 1.75 2^8, s = 2^(E - 8) when m <= 1.75, else 2^(E - 7).  The floor
+    2^-126 (reading: the page gives no range) keeps s and 1/s float32 normals.
     """
     a = np.asarray(amax, dtype=np.float64)
     if np.any(~np.isfinite(a)) or np.any(a < 0):
         raise ValueError("amax must be finite and >= 0")
     m, e = np.frexp(a)             # a = m 2^e, m in [0.5, 1)
     mant, E = 2.0 * m, e - 1       # a = mant 2^E, mant in [1, 2)
-    exp = np.where(mant <= 1.75, E - 8, E - 7)
+    exp = np.maximum(np.where(mant <= 1.75, E - 8, E - 7), -126)
     s = np.where(a > 0, np.ldexp(1.0, exp), 1.0)
     return s.astype(np.float32)
 

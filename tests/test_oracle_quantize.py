@@ -89,6 +89,9 @@ def test_block_scale_rule():
         assert Qz.block_scale(np.nextafter(a, np.inf)) == np.float32(2.0 ** (e + 1))
         assert Qz.block_scale(np.nextafter(a, 0)) == np.float32(2.0 ** e)
     assert Qz.block_scale(0.0) == 1.0
+    # the floor: tiny blocks get 2^-126, and then amax / s < 224
+    assert Qz.block_scale(448.0 * 2.0 ** -127) == np.float32(2.0 ** -126)
+    assert Qz.block_scale(1e-40) == np.float32(2.0 ** -126)
     rng = np.random.default_rng(5)
     amax = np.exp(rng.uniform(-30, 30, 10000))
     s = Qz.block_scale(amax).astype(np.float64)
