@@ -96,6 +96,47 @@ int fp8attn_pzero_count(const void* q, const void* k, const void* v,
                         float p_scale, int kv_order, int n_sink, void* stream);
 
 /*
+ * Quantisation in front of the attention path ("Attenzione flash e domanda
+ * sulla lunghezza della sequenza", section "FA3: Meccanica della tramoggia",
+ * point 3: block quantisation to FP8, after a random rotation that spreads
+ * outlier channels over all coordinates).
+ *
+ * x is a device array [Z, N, d] of bfloat16 (x_dtype = 0) or float32
+ * (x_dtype = 1), contiguous, 16-byte aligned, finite.  Each row is optionally
+ * rotated by R = diag(signs) H_d / sqrt(d) (H_d the Sylvester Hadamard
+ * matrix; signs is a HOST array of d values, each +1 or -1, read during the
+ * call; NULL = no rotation), evaluated as the radix-2 fast transform in
+ * float32.  Rows are then cast to E4M3 (xq: device [Z, N, d], 16-byte
+ * aligned) with one descale per block: the smallest power of two s >= 2^-126
+ * with max|x| <= 448 s, so that x = s * E4M3 code up to the cast's rounding
+ * and nothing saturates.  Blocks are block_rows (1..128) consecutive rows of
+ * one slab, scales is then a device float array [Z, ceil(N / block_rows)];
+ * block_rows = 0 gives one descale per slab, scales [Z] (three launches; the
+ * array holds intermediate maxima until the last one).  d must be 64 or 128.
+ * For fp8attn_fwd_scaled: Q and K with block_rows = 128, V with 0, the same
+ * signs for all three.
+ */
+int fp8attn_quantize(const void* x, int x_dtype, void* xq, float* scales,
+                     int Z, int N, int d, int block_rows, const float* signs, void* stream);
+
+/*
+ * Forward pass on quantised inputs: q = q_scales * q codes per 128-row query
+ * tile ([B * H, ceil(N / 128)]), k = k_scales * k codes per 128-key tile
+ * ([B * Hkv, ceil(N / 128)]), v = v_scales * v codes per head ([B * Hkv]),
+ * all scales device float arrays (powers of two as fp8attn_quantize writes
+ * them).  The P-cast, orders, masks and outputs are those of fp8attn_fwd on
+ * the descaled values; when signs (HOST, d values of +-1, the ones used to
+ * quantize) is not NULL, each output row is rotated back by R^T before the
+ * bfloat16 rounding, so o is the attention of the unrotated inputs.  d must
+ * be 128 (FP8ATTN_ERR_UNSUPPORTED otherwise).  The scratch is that of
+ * fp8attn_fwd.
+ */
+int fp8attn_fwd_scaled(const void* q, const void* k, const void* v, void* o, float* lse,
+                       const float* q_scales, const float* k_scales, const float* v_scales,
+                       const float* signs, int B, int H, int Hkv, int N, int d, int causal,
+                       float p_scale, int kv_order, void* stream);
+
+/*
  * Allocation-free forward pass.  The pages have no counterpart of this call:
  * it is an interface for callers that cannot let the library allocate device
  * memory -- programs that hand the whole device memory to their own allocator

@@ -15,6 +15,7 @@
 #include "../../include/fp8attn.h"
 #include "fwd_v1.cuh"
 #include "fwd_v2.cuh"
+#include "quantize.cuh"
 
 namespace fp8attn {
 
@@ -65,6 +66,21 @@ bool make_map(CUtensorMap* map, const void* ptr, int D, int rows, int Z, int box
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Packs host signs (d values of +-1) into bit words: bit i set for -1.
+// Returns false if a value is not +-1.
+bool pack_signs(const float* signs, int d, uint32_t (&bits)[4]) {
+  bits[0] = bits[1] = bits[2] = bits[3] = 0u;
+  for (int i = 0; i < d; ++i) {
+    if (signs[i] == -1.0f) {
+      bits[i >> 5] |= 1u << (i & 31);
+    } else if (signs[i] != 1.0f) {
+      return false;
+    }
+  }
+  return true;
+}
+
+
 int validate(const void* q, const void* k, const void* v, int B, int H, int Hkv, int N, int d, float p_scale,
              int kv_order) {
   if (B < 0 || N < 0 || H < 1 || Hkv < 1 || H % Hkv != 0) return FP8ATTN_ERR_INVALID_ARG;
@@ -114,14 +130,14 @@ int num_sms() {
 }
 
 // Persistent warp-specialised kernel (d = 128): one CTA per SM.
-template <bool COUNT>
+template <bool COUNT, bool SCALED = false>
 int launch_v2(const void* q, const void* k, const void* v, FwdParams p, cudaStream_t stream) {
   using C = V2Config;
   CUtensorMap tq, tk, tv;
   if (!make_map(&tq, q, 128, p.N, p.B * p.H, 128) || !make_map(&tk, k, 128, p.N, p.B * p.Hkv, 128) ||
       !make_map(&tv, v, 128, p.N, p.B * p.Hkv, 128))
     return FP8ATTN_ERR_CUDA;
-  auto kern = fwd_v2_kernel<COUNT>;
+  auto kern = fwd_v2_kernel<COUNT, SCALED>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return FP8ATTN_ERR_CUDA;
   // The warpgroups re-split the block's registers with setmaxnreg; that split
@@ -308,6 +324,30 @@ extern "C" int fp8attn_pzero_count(const void* q, const void* k, const void* v, 
   return d == 128 ? launch_v2<true>(q, k, v, p, s) : launch<64, true>(q, k, v, p, s);
 }
 
+extern "C" int fp8attn_fwd_scaled(const void* q, const void* k, const void* v, void* o, float* lse,
+                                  const float* q_scales, const float* k_scales, const float* v_scales,
+                                  const float* signs, int B, int H, int Hkv, int N, int d, int causal, float p_scale,
+                                  int kv_order, void* stream) {
+  int st = validate(q, k, v, B, H, Hkv, N, d, p_scale, kv_order);
+  if (st != FP8ATTN_OK) return st;
+  if (d != 128) return FP8ATTN_ERR_UNSUPPORTED;
+  FwdParams p = base_params(B, H, Hkv, N, causal, p_scale, kv_order);
+  if (signs != nullptr) {
+    if (!pack_signs(signs, d, p.sign_bits)) return FP8ATTN_ERR_INVALID_ARG;
+    p.unrotate = 1;
+  }
+  if (static_cast<int64_t>(B) * H * N == 0) return FP8ATTN_OK;
+  if (!o || !aligned16(o) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))) return FP8ATTN_ERR_INVALID_ARG;
+  auto aligned4 = [](const void* ptr) { return ptr != nullptr && (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; };
+  if (!aligned4(q_scales) || !aligned4(k_scales) || !aligned4(v_scales)) return FP8ATTN_ERR_INVALID_ARG;
+  p.o = o;
+  p.lse = lse;
+  p.q_scales = q_scales;
+  p.k_scales = k_scales;
+  p.v_scales = v_scales;
+  return launch_v2<false, true>(q, k, v, p, static_cast<cudaStream_t>(stream));
+}
+
 extern "C" int fp8attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
                                    int Hkv, int N, int d, int causal, float p_scale, int kv_order, void* stream) {
   int st = validate(q, k, v, B, H, Hkv, N, d, p_scale, kv_order);
@@ -324,6 +364,61 @@ extern "C" int fp8attn_fwd_noalloc(const void* q, const void* k, const void* v, 
   p.lse = lse;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 128 ? launch_v2_noalloc(q, k, v, p, s, *dev) : launch<64, false>(q, k, v, p, s);
+}
+
+namespace fp8attn {
+namespace {
+
+template <int E>
+int launch_quantize(QuantParams p, cudaStream_t s) {
+  const dim3 block(kQuantWarps * 32);
+  if (p.block_rows > 0) {
+    const dim3 grid((p.N + p.block_rows - 1) / p.block_rows, p.Z);
+    if (grid.x > 0) quantize_kernel<E, 0><<<grid, block, 0, s>>>(p);
+  } else {
+    if (cudaMemsetAsync(p.scales, 0, sizeof(float) * static_cast<size_t>(p.Z), s) != cudaSuccess)
+      return FP8ATTN_ERR_CUDA;
+    p.block_rows = 128;
+    const dim3 grid((p.N + 127) / 128, p.Z);
+    if (grid.x > 0) {
+      quantize_kernel<E, 1><<<grid, block, 0, s>>>(p);
+      quantize_kernel<E, 2><<<grid, block, 0, s>>>(p);
+    }
+    quantize_finish_kernel<<<(p.Z + 255) / 256, 256, 0, s>>>(p.scales, p.Z);
+  }
+  return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace fp8attn
+
+extern "C" int fp8attn_quantize(const void* x, int x_dtype, void* xq, float* scales, int Z, int N, int d,
+                                int block_rows, const float* signs, void* stream) {
+  if (Z < 0 || N < 0 || (d != 64 && d != 128) || (x_dtype != 0 && x_dtype != 1) || block_rows < 0 ||
+      block_rows > 128)
+    return (d != 64 && d != 128) ? FP8ATTN_ERR_UNSUPPORTED : FP8ATTN_ERR_INVALID_ARG;
+  if (Z > 65535) return FP8ATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(Z) * N * d > (int64_t(1) << 40)) return FP8ATTN_ERR_UNSUPPORTED;
+  QuantParams p;
+  std::memset(&p, 0, sizeof(p));
+  if (signs != nullptr) {
+    if (!pack_signs(signs, d, p.sign_bits)) return FP8ATTN_ERR_INVALID_ARG;
+    p.rotate = 1;
+  }
+  if (Z == 0 || (N == 0 && block_rows > 0)) return FP8ATTN_OK;
+  if (!scales || (reinterpret_cast<uintptr_t>(scales) & 3u)) return FP8ATTN_ERR_INVALID_ARG;
+  if (N > 0 && (!x || !xq || !aligned16(x) || !aligned16(xq))) return FP8ATTN_ERR_INVALID_ARG;
+  p.x = x;
+  p.xq = static_cast<uint8_t*>(xq);
+  p.scales = scales;
+  p.Z = Z;
+  p.N = N;
+  p.d = d;
+  p.block_rows = block_rows;
+  p.nblocks = block_rows > 0 ? (N + block_rows - 1) / block_rows : 1;
+  p.x_f32 = x_dtype;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 128 ? launch_quantize<32>(p, s) : launch_quantize<16>(p, s);
 }
 
 extern "C" int fp8attn_kv_tile(int d) {

@@ -37,6 +37,13 @@ struct FwdParams {
   float p_scale;                // S
   float scale_log2;             // log2(e) / sqrt(D)
   float log2_p_scale;           // log2(S), rounded to float
+  // Descaled inputs (persistent kernel, SCALED instance only): q = q_scale *
+  // E4M3 codes per 128-row query tile, k likewise per key tile, v per head.
+  const float* q_scales;        // [B * H, num_q_tiles]
+  const float* k_scales;        // [B * Hkv, num_kv_tiles]
+  const float* v_scales;        // [B * Hkv]
+  int unrotate;                 // rotate each output row back by R^T = H_D diag(signs) / sqrt(D)
+  uint32_t sign_bits[4];        // bit i set: signs[i] = -1
 };
 
 template <int D>

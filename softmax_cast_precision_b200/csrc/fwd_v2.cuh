@@ -159,7 +159,10 @@ constexpr uint32_t kUnitReaders = 2 + 256;
 // Pairs out of every eight (16 keys) whose exponentials use the polynomial.
 constexpr int kPolyPairs = 2;
 
-template <bool COUNT>
+// SCALED: the inputs carry descales (FwdParams q/k/v_scales) and optionally
+// a rotation to undo on the output; the running maximum is then kept in
+// log2 units of the descaled logits, whose scale changes from tile to tile.
+template <bool COUNT, bool SCALED = false>
 __global__ void __launch_bounds__(V2Config::THREADS, 1)
     fwd_v2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p, uint32_t* err_word) {
@@ -407,7 +410,11 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
       uint32_t prev_cnt = 2;
       const int qk = g.q0 + 128 * k;
       const int row = qk + r;
-      float m = -INFINITY;  // running max of raw logits
+      // Running maximum: of the raw logits, or for SCALED inputs of the
+      // descaled logits in log2 units (x = s * c_t with a per-tile c_t).
+      float m = -INFINITY;
+      float c_q = p.scale_log2;  // log2(e) / sqrt(d), times the query tile's descale when SCALED
+      if constexpr (SCALED) c_q *= p.q_scales[static_cast<int64_t>(g.zq) * p.num_q_tiles + (qk >> 7)];
       float l = 0.0f;
       uint32_t nzero = 0;
       int j = 0;
@@ -415,6 +422,8 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         const int t = stream_tile(p, g, idx);
         if (t > last) continue;
         const int j0 = t * 128;
+        float c_t = c_q;  // scale of this tile's logits into log2 units
+        if constexpr (SCALED) c_t *= __ldg(p.k_scales + static_cast<int64_t>(g.zkv) * p.num_kv_tiles + t);
         ok = __all_sync(0xffffffffu, v2_wait(bars, &bars->s_full[k], s_it & 1, err_word, kErrTimeoutMMA));
         if (!ok) break;  // warp-uniform, so the collective TMEM loads below stay converged
         ++s_it;
@@ -450,7 +459,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
           float h1[22];
 #pragma unroll
           for (int i = 0; i < 21; ++i) h1[i] = fmax3(s[3 * i], s[3 * i + 1], s[3 * i + 2]);
-          h1[21] = fmaxf(s[63], m);
+          h1[21] = SCALED ? s[63] : fmaxf(s[63], m);
           float h2[8];
 #pragma unroll
           for (int i = 0; i < 7; ++i) h2[i] = fmax3(h1[3 * i], h1[3 * i + 1], h1[3 * i + 2]);
@@ -486,7 +495,8 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
           t2[7] = t1[21];
           m_new = fmaxf(fmax3(fmax3(t2[0], t2[1], t2[2]), fmax3(t2[3], t2[4], t2[5]), t2[6]), t2[7]);
         }
-        const float ms = (m_new == -INFINITY) ? 0.0f : m_new * p.scale_log2;
+        if constexpr (SCALED) m_new = fmaxf(m_new * c_t, m);
+        const float ms = (m_new == -INFINITY) ? 0.0f : (SCALED ? m_new : m_new * p.scale_log2);
         // P * S = 2^(x - m_new + log2 S) with x = s * log2(e) / sqrt(d)
         // (packed pairs): the scale enters the exponent, so one exponential
         // gives the scaled probability.  Its row sum, l * S, is kept (eight
@@ -494,7 +504,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         // goes straight to the P buffer this tile uses (its previous reader,
         // the P V product two tiles back, is known to be complete).
         const uint32_t sPb = sPk + (p_cnt & 1) * C::TILE_BYTES;
-        const uint64_t sc2 = f2_pack(p.scale_log2, p.scale_log2);
+        const uint64_t sc2 = f2_pack(c_t, c_t);
         const float bias = p.log2_p_scale - ms;
         const uint64_t nm2 = f2_pack(bias, bias);
         uint64_t acc[8];
@@ -550,7 +560,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         // change (the product m * c is then not recomputed), 0 before the
         // first visible key.  Formed after the exponentials so that this one
         // MUFU operation never waits behind them.
-        const float alpha = (m_new == m) ? 1.0f : ex2_approx(fmaf(m, p.scale_log2, -ms));
+        const float alpha = (m_new == m) ? 1.0f : ex2_approx(SCALED ? m - ms : fmaf(m, p.scale_log2, -ms));
         l = l * alpha + rowsum;  // l * S
         m = m_new;
 
@@ -600,8 +610,48 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         const uint32_t total = __reduce_add_sync(0xffffffffu, nzero);
         if (lane == 0 && total) atomicAdd(p.counts + g.zq, static_cast<unsigned long long>(total));
       } else {
-        const float inv = __frcp_rn(l);  // l holds l * S
+        float inv = __frcp_rn(l);  // l holds l * S
+        if constexpr (SCALED) inv *= p.v_scales[g.zkv];
         uint8_t* orow = static_cast<uint8_t*>(p.o) + ((static_cast<int64_t>(g.zq) * p.N + row) * 128) * 2;
+        if (SCALED && p.unrotate) {
+          // O_row R^T: the Walsh-Hadamard transform of the whole row (radix-2
+          // stages of half-width 1, 2, ..., 64, sum first), times
+          // float32(1/sqrt(128)), then the signs.
+          float y[128];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t rr[32];
+            tmem_ld32(tO + c * 32, rr);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) y[c * 32 + i] = __uint_as_float(rr[i]);
+          }
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 128; ++i) y[i] *= inv;
+#pragma unroll
+          for (int h = 1; h < 128; h *= 2) {
+#pragma unroll
+            for (int i = 0; i < 128; ++i) {
+              if ((i & h) == 0) {
+                const float a = y[i], b = y[i + h];
+                y[i] = a + b;
+                y[i + h] = a - b;
+              }
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 128; ++i) {
+            const float t = y[i] * 0.08838834764831845f;  // float32(1/sqrt(128))
+            y[i] = ((p.sign_bits[i >> 5] >> (i & 31)) & 1u) ? -t : t;
+          }
+          if (row < p.N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              dst[i] = make_uint4(pack_bf16x2(y[8 * i], y[8 * i + 1]), pack_bf16x2(y[8 * i + 2], y[8 * i + 3]),
+                                  pack_bf16x2(y[8 * i + 4], y[8 * i + 5]), pack_bf16x2(y[8 * i + 6], y[8 * i + 7]));
+          }
+        } else {
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t rr[32];
@@ -617,9 +667,10 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
             for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
           }
         }
+        }
         if (p.lse != nullptr && row < p.N)
           p.lse[static_cast<int64_t>(g.zq) * p.N + row] =
-              (m * p.scale_log2 + (log2f(l) - p.log2_p_scale)) * 0.6931471805599453f;
+              ((SCALED ? m : m * p.scale_log2) + (log2f(l) - p.log2_p_scale)) * 0.6931471805599453f;
       }
       tc_fence_before();
       mbar_arrive(&bars->o_free[k]);

@@ -12,6 +12,7 @@ float32.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import threading
 
@@ -51,6 +52,10 @@ def lib() -> ctypes.CDLL:
         L.fp8attn_fwd.restype = i32
         L.fp8attn_fwd_noalloc.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, P]
         L.fp8attn_fwd_noalloc.restype = i32
+        L.fp8attn_quantize.argtypes = [P, i32, P, P, i32, i32, i32, i32, P, P]
+        L.fp8attn_quantize.restype = i32
+        L.fp8attn_fwd_scaled.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, P]
+        L.fp8attn_fwd_scaled.restype = i32
         L.fp8attn_pzero_count.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, P]
         L.fp8attn_pzero_count.restype = i32
         L.fp8attn_kv_tile.argtypes = [i32]
@@ -175,6 +180,76 @@ def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Te
                                    _stream_ptr(q.device, stream))
     if st != OK:
         raise Fp8AttnError(st, "fp8attn_fwd_noalloc")
+
+
+def _host_signs(signs, d: int):
+    """Signs as a host float32 array kept alive for the call (None -> NULL)."""
+    if signs is None:
+        return None, ctypes.c_void_p(0)
+    a = torch.as_tensor(signs, dtype=torch.float32).detach().cpu().contiguous().reshape(-1)
+    if a.numel() != d:
+        raise ValueError(f"signs must have {d} entries")
+    return a, ctypes.c_void_p(a.data_ptr())
+
+
+def quantize(x: torch.Tensor, block_rows: int, signs=None, *, out: torch.Tensor | None = None,
+             scales: torch.Tensor | None = None, stream=None):
+    """E4M3 codes and per-block descales of x [..., N, d] (bfloat16 or float32, on the GPU).
+
+    Rows are rotated by R = diag(signs) H_d / sqrt(d) first when ``signs``
+    (d values of +-1) is given.  ``block_rows`` rows of one slab share a
+    descale (0: one per slab).  Returns (codes uint8 of x's shape, scales
+    float32 [Z, nblocks]) with Z the product of the leading dimensions.
+    """
+    if not x.is_cuda:
+        raise ValueError("quantize takes a device tensor")
+    if x.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("x must be bfloat16 or float32")
+    x = x.contiguous()
+    N, d = int(x.shape[-2]), int(x.shape[-1])
+    Z = math.prod(int(n) for n in x.shape[:-2])
+    nb = 1 if block_rows == 0 else -(-N // block_rows)
+    codes = out if out is not None else torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    sc = scales if scales is not None else torch.empty((Z, nb), dtype=torch.float32, device=x.device)
+    keep, sp = _host_signs(signs, d)
+    st = lib().fp8attn_quantize(_ptr(x), 0 if x.dtype == torch.bfloat16 else 1, _ptr(codes), _ptr(sc), Z, N, d,
+                                int(block_rows), sp, _stream_ptr(x.device, stream))
+    del keep
+    if st != OK:
+        raise Fp8AttnError(st, "fp8attn_quantize")
+    return codes, sc
+
+
+def fwd_scaled(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_scales: torch.Tensor, k_scales: torch.Tensor,
+               v_scales: torch.Tensor, *, causal: bool, p_scale: float = 256.0, kv_order="reverse", signs=None,
+               with_lse: bool = True, stream=None):
+    """Forward pass on quantised q, k, v (E4M3 codes) with their descales; see fp8attn_fwd_scaled."""
+    q, k, v = _bytes(q), _bytes(k), _bytes(v)
+    B, H, Hkv, N, d = _shapes(q, k, v)
+    if not q.is_cuda:
+        raise ValueError("fwd_scaled takes device tensors")
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if with_lse else None
+    qs, ks, vs = (t.contiguous().float() for t in (q_scales, k_scales, v_scales))
+    keep, sp = _host_signs(signs, d)
+    st = lib().fp8attn_fwd_scaled(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(qs), _ptr(ks), _ptr(vs), sp,
+                                  B, H, Hkv, N, d, int(bool(causal)), ctypes.c_float(p_scale), _order(kv_order),
+                                  _stream_ptr(q.device, stream))
+    del keep
+    if st != OK:
+        raise Fp8AttnError(st, "fp8attn_fwd_scaled")
+    return o, lse
+
+
+def fwd_wide(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_scale: float = 256.0,
+             kv_order="reverse", signs=None, with_lse: bool = True, stream=None):
+    """Attention on bfloat16/float32 q [B,H,N,d], k, v [B,Hkv,N,d]: quantise (Q, K per 128-row
+    block, V per head, rotated by ``signs`` when given), then the scaled forward pass."""
+    qc, qs = quantize(q, 128, signs, stream=stream)
+    kc, ks = quantize(k, 128, signs, stream=stream)
+    vc, vs = quantize(v, 0, signs, stream=stream)
+    return fwd_scaled(qc, kc, vc, qs, ks, vs, causal=causal, p_scale=p_scale, kv_order=kv_order, signs=signs,
+                      with_lse=with_lse, stream=stream)
 
 
 def pzero_count(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_scale: float = 256.0,

@@ -30,7 +30,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for required in ["fp8attn_fwd", "fp8attn_fwd_noalloc", "fp8attn_pzero_count", "fp8attn_kv_tile", "fp8attn_status_str",
+    for required in ["fp8attn_fwd", "fp8attn_fwd_noalloc", "fp8attn_fwd_scaled", "fp8attn_quantize",
+                     "fp8attn_pzero_count", "fp8attn_kv_tile", "fp8attn_status_str",
                      "fp8attn_check_error"]:
         assert required in names
 
@@ -116,3 +117,42 @@ def test_binding_raises_without_fallback(fp8, monkeypatch):
     monkeypatch.setattr(mod, "LIB_PATH", "/nonexistent/libfp8attn.so")
     with pytest.raises(RuntimeError, match="no fallback"):
         mod.lib()
+
+
+def _call_quantize(fp8, x=16, dtype=0, xq=16, scales=16, Z=2, N=300, d=128, block_rows=128, signs=None):
+    P = ctypes.c_void_p
+    sp = P(0)
+    keep = None
+    if signs is not None:
+        keep = (ctypes.c_float * len(signs))(*signs)
+        sp = ctypes.cast(keep, P)
+    return fp8.lib().fp8attn_quantize(P(x), dtype, P(xq), P(scales), Z, N, d, block_rows, sp, P(0))
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(d=96), 2), (dict(d=256), 2), (dict(dtype=2), 1), (dict(block_rows=-1), 1), (dict(block_rows=129), 1),
+    (dict(Z=-1), 1), (dict(N=-1), 1), (dict(x=0), 1), (dict(x=8), 1), (dict(xq=8), 1), (dict(scales=0), 1),
+    (dict(scales=2), 1), (dict(Z=70000), 2), (dict(signs=[1.0] * 127 + [0.5]), 1),
+    (dict(Z=0), 0), (dict(N=0), 0), (dict(N=0, x=0, xq=0), 0),
+])
+def test_quantize_validation(fp8, kw, expected):
+    assert _call_quantize(fp8, **kw) == expected
+
+
+def _call_fwd_scaled(fp8, qs=16, ks=16, vs=16, d=128, signs=None, N=128, S=256.0):
+    P = ctypes.c_void_p
+    sp = P(0)
+    keep = None
+    if signs is not None:
+        keep = (ctypes.c_float * len(signs))(*signs)
+        sp = ctypes.cast(keep, P)
+    return fp8.lib().fp8attn_fwd_scaled(P(16), P(16), P(16), P(16), P(0), P(qs), P(ks), P(vs), sp, 1, 2, 1, N, d, 1,
+                                        ctypes.c_float(S), 1, P(0))
+
+
+@pytest.mark.parametrize("kw,expected", [
+    (dict(d=64), 2), (dict(d=96), 2), (dict(qs=0), 1), (dict(ks=2), 1), (dict(vs=0), 1), (dict(S=0.0), 1),
+    (dict(signs=[1.0, -1.0] * 63 + [2.0, 1.0]), 1), (dict(N=0, qs=0, ks=0, vs=0), 0),
+])
+def test_fwd_scaled_validation(fp8, kw, expected):
+    assert _call_fwd_scaled(fp8, **kw) == expected
