@@ -1,6 +1,6 @@
 """Throughput benchmark of the FP8 (E4M3) P-cast attention forward pass.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--path fp8|wide]
 
 One step is one forward pass of the 32K causal prefill (B=1, H=32, N=32768,
 d=128, Delta=7 sink with k=4, S=256, reverse KV order) through the C ABI.
@@ -10,6 +10,10 @@ the data path: weak scaling); the step time is the maximum over ranks.
 
 --impl reference times the CPU oracle (the blockwise E4M3 emulator) on the
 host cores instead, on a bounded sample of the same workload per step.
+
+--path wide starts from bfloat16 Q, K, V instead: one step quantises them
+(random-sign Hadamard rotation, Q and K per 128-row block, V per head) and
+runs the scaled forward pass, which rotates the output back.
 """
 from __future__ import annotations
 
@@ -54,6 +58,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--path", default="fp8", choices=["fp8", "wide"],
+                    help="fp8: E4M3 inputs (the headline); wide: bfloat16 inputs quantised in the step")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (used under ncu)")
     return ap.parse_args()
@@ -232,6 +238,225 @@ def mse_vs_fp64(qd, kd, vd, o, rows_np):
     return float(((o[:, :, rows].double() - ref) ** 2).mean().item())
 
 
+WIDE_WORKLOAD_DESC = ("prefill32k from bfloat16: B=1 H=32 N=32768 d=128 causal, Delta=7 sink (k=4); Q/K/V quantised "
+                      "to E4M3 in the step (random-sign Hadamard rotation, Q/K per 128-row block, V per head), "
+                      "S=256, reverse KV order, output rotated back")
+WIDE_CPU_ROWS = 512
+
+
+def wide_inputs(seed: int):
+    w = WORKLOAD
+    q, k, v, _ = synthetic.make_wide_inputs(w.B, w.H, w.Hkv, w.N, w.d, w.delta, seed=seed, n_sink=w.n_sink)
+    return q, k, v, synthetic.hadamard_signs(w.d, seed + 7)
+
+
+def cpu_wide_run(q, k, v, signs, rows):
+    """One bounded step of the oracle on the wide path: quantise all of Q, K, V,
+    then the emulator on `rows` of every head and the inverse rotation."""
+    from oracle import quantize as Qz
+
+    w = WORKLOAD
+    t0 = time.perf_counter()
+    Qz.quantized_attention(q, k, v, signs, causal=w.causal, p_scale=P_SCALE, reverse=bool(KV_ORDER), rows=rows)
+    dt = time.perf_counter() - t0
+    return 4.0 * w.d * visible_pairs(rows, w.N, w.causal) * w.B * w.H, dt
+
+
+def run_wide(args, rank, world, local_rank):
+    """The wide path: quantise bfloat16 inputs, then the scaled forward pass."""
+    import torch
+
+    from softmax_cast_precision_b200 import fp8attn
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    w = WORKLOAD
+    q, k, v, signs = wide_inputs(rank_seed(rank))
+    qb, kb, vb = (torch.from_numpy(x).to(device).to(torch.bfloat16) for x in (q, k, v))
+    stream = torch.cuda.current_stream(device)
+    ev_q0, ev_q1, ev_f1 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    quant_ms, fwd_ms = [], []
+
+    def step(timed=False):
+        if timed:
+            ev_q0.record(stream)
+        qc, qs = fp8attn.quantize(qb, 128, signs, stream=stream)
+        kc, ks = fp8attn.quantize(kb, 128, signs, stream=stream)
+        vc, vs = fp8attn.quantize(vb, 0, signs, stream=stream)
+        if timed:
+            ev_q1.record(stream)
+        o, lse = fp8attn.fwd_scaled(qc, kc, vc, qs, ks, vs, causal=w.causal, p_scale=P_SCALE, kv_order=KV_ORDER,
+                                    signs=signs, stream=stream)
+        if timed:
+            ev_f1.record(stream)
+            ev_f1.synchronize()
+            quant_ms.append(ev_q0.elapsed_time(ev_q1))
+            fwd_ms.append(ev_q1.elapsed_time(ev_f1))
+        return o, lse
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    fp8attn.check_error(stream=stream, device=device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize(device)
+        ev[0].record(stream)
+        for i in range(args.steps):
+            o, lse = step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+    fp8attn.check_error(stream=stream, device=device)
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), dist, device)
+    ms_per_step = total_ms / args.steps
+    flops = w.flops()
+    # Per-kernel durations, from separately synchronised steps after the timed region.
+    for _ in range(5):
+        step(timed=True)
+
+    # End to end: bfloat16 inputs from pinned host memory, outputs back.
+    qh, kh, vh = (t.cpu().pin_memory() for t in (qb, kb, vb))
+    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    qd, kd, vd = (torch.empty_like(t) for t in (qb, kb, vb))
+
+    def e2e_step():
+        for dst, src in ((qd, qh), (kd, kh), (vd, vh)):
+            dst.copy_(src, non_blocking=True)
+        oo, ll = fp8attn.fwd_wide(qd, kd, vd, causal=w.causal, p_scale=P_SCALE, kv_order=KV_ORDER, signs=signs,
+                                  stream=stream)
+        oh.copy_(oo, non_blocking=True)
+        lh.copy_(ll, non_blocking=True)
+
+    e2e_step()
+    e2e_steps = max(3, min(args.steps, 10))
+    barrier()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, device)
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+    mse = None
+    if rank == 0:
+        rows = sample_rows(w.N, 256)
+        mse = wide_mse_vs_fp64(qb, kb, vb, o, rows)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peak_burst, peak_sustained, peak_src = fp8_peak()
+    fwd_kernel_ms = statistics.mean(fwd_ms)
+    quant_kernel_ms = statistics.mean(quant_ms)
+    achieved = flops / (fwd_kernel_ms * 1e-3) / 1e12
+    hbm = hbm_peak()
+    quant_bytes = 3 * (qb.numel() * 3)  # three tensors, 2 B read + 1 B written per element
+    line = {
+        "metric": METRIC, "value": aggregate_throughput(flops, world, ms_per_step), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3", "data": "synthetic",
+        "config": {"workload": WIDE_WORKLOAD_DESC, "flop_per_step_per_gpu": flops,
+                   "l2": "inputs exceed L2 (805 MB bfloat16)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "gpu_launches": 6 * args.steps,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_burst, "unit": "TFLOP/s",
+                     "frac": achieved / peak_burst, "traffic": None,
+                     "peak_source": f"{peak_src}: bf16 cuBLAS burst x {FP8_OVER_BF16} (FP8/BF16 nominal)",
+                     "kernel": "fwd_v2_kernel<0,1> (scaled)", "kernel_ms": fwd_kernel_ms},
+        "roofline_quantize": {"bound": "hbm", "achieved": quant_bytes / (quant_kernel_ms * 1e-3) / 1e9,
+                              "peak": hbm, "unit": "GB/s",
+                              "frac": quant_bytes / (quant_kernel_ms * 1e-3) / 1e9 / hbm,
+                              "algorithmic_bytes": quant_bytes, "ms": quant_kernel_ms,
+                              "note": "3 tensors x (2 B read + 1 B written) per element; V's per-head descale "
+                                      "reads V twice"},
+        "e2e": {"value": aggregate_throughput(flops, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "clocks": clk.summary(),
+        "mse_vs_fp64": {"value": mse, "rows": "256 evenly spaced query rows of each head",
+                        "reference": "PyTorch float64 softmax(QK^T/sqrt(d))V on the bfloat16 inputs"},
+    }
+    if not args.skip_cpu_baseline:
+        import oracle
+
+        rows = sample_rows(w.N, WIDE_CPU_ROWS)
+        f, dt = cpu_wide_run(q, k, v, signs, rows)
+        line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                                "sample": f"quantisation of all of Q, K, V, then the emulator on {len(rows)} evenly "
+                                          f"spaced query rows of each head ({f / 1e12:.3f} TFLOP in {dt:.1f} s)"}
+    print(json.dumps(line), flush=True)
+
+
+def hbm_peak() -> float:
+    try:
+        with open(PEAKS_FILE) as fh:
+            return float(json.load(fh)["hbm_gbs"])
+    except (OSError, KeyError, ValueError):
+        return 6650.0
+
+
+def wide_mse_vs_fp64(qb, kb, vb, o, rows_np):
+    """MSE of the output against FP64 attention on the bfloat16 inputs, over the given rows."""
+    import torch
+
+    w = WORKLOAD
+    rows = torch.from_numpy(rows_np.astype(np.int64)).to(qb.device)
+    qf = qb[:, :, rows].double()
+    kf, vf = kb.double(), vb.double()
+    rep = w.H // w.Hkv
+    kf, vf = kf.repeat_interleave(rep, 1), vf.repeat_interleave(rep, 1)
+    s = qf @ kf.transpose(-1, -2) / math.sqrt(w.d)
+    if w.causal:
+        keys = torch.arange(w.N, device=qb.device)
+        s = s.masked_fill(keys[None, None, None, :] > rows[None, None, :, None], float("-inf"))
+    ref = torch.softmax(s, -1) @ vf
+    return float(((o[:, :, rows].double() - ref) ** 2).mean().item())
+
+
+def run_reference_wide(args, rank):
+    """The oracle arm of the wide path (rank 0 only)."""
+    if rank != 0:
+        return
+    import oracle
+
+    q, k, v, signs = wide_inputs(SEED)
+    rows = sample_rows(WORKLOAD.N, 64)
+    for _ in range(args.warmup):
+        cpu_wide_run(q[:, :, :256], k[:, :, :256], v[:, :, :256], signs, rows[:2] // 128)
+    total_flops, total_t = 0.0, 0.0
+    for _ in range(args.steps):
+        f, dt = cpu_wide_run(q, k, v, signs, rows)
+        total_flops += f
+        total_t += dt
+    value = total_flops / total_t / 1e12
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16->e4m3/f32",
+        "data": "synthetic", "config": {"workload": WIDE_WORKLOAD_DESC, "l2": "inputs exceed L2"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"per step: quantisation of all of Q, K, V and the emulator on {len(rows)} "
+                                   "evenly spaced query rows of each head"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
 def run_reference(args, rank, world):
     """The oracle arm: emulator steps on the host cores (rank 0 only)."""
     if rank != 0:
@@ -269,7 +494,9 @@ def main():
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
-        return run_reference(args, rank, world)
+        return run_reference_wide(args, rank) if args.path == "wide" else run_reference(args, rank, world)
+    if args.path == "wide":
+        return run_wide(args, rank, world, local_rank)
 
     import torch
 
