@@ -137,6 +137,21 @@ int fp8attn_fwd_scaled(const void* q, const void* k, const void* v, void* o, flo
                        float p_scale, int kv_order, void* stream);
 
 /*
+ * Forward pass with bfloat16 Q and K: q [B, H, N, d] and k [B, Hkv, N, d]
+ * bfloat16, v [B, Hkv, N, d] E4M3 (device, contiguous, 16-byte aligned).
+ * S = Q K^T runs on the tensor cores' 16-bit path with FP32 accumulation;
+ * the running maximum, the P-cast E4M3(P * S), P^ V in FP8 and the epilogue
+ * are those of fp8attn_fwd.  This is the setting of the P-cast summary's
+ * kernel-faithful experiments, which keep Q and K in high precision to
+ * isolate the cast of P ("P-Cast Precision in FP8 Attention", section 3,
+ * point 4, and section 4).  d must be 128
+ * (FP8ATTN_ERR_UNSUPPORTED otherwise); the scratch is that of fp8attn_fwd.
+ */
+int fp8attn_fwd_bf16qk(const void* q, const void* k, const void* v, void* o, float* lse,
+                       int B, int H, int Hkv, int N, int d, int causal,
+                       float p_scale, int kv_order, void* stream);
+
+/*
  * Allocation-free forward pass.  The pages have no counterpart of this call:
  * it is an interface for callers that cannot let the library allocate device
  * memory -- programs that hand the whole device memory to their own allocator

@@ -64,6 +64,21 @@ bool make_map(CUtensorMap* map, const void* ptr, int D, int rows, int Z, int box
   return r == CUDA_SUCCESS;
 }
 
+// A [Z, rows, 128] bfloat16 tensor read in boxes of 128 rows x 64 columns
+// (one 128-byte swizzle panel per box; a 128 x 128 tile takes two boxes).
+bool make_map_bf16(CUtensorMap* map, const void* ptr, int rows, int Z) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(Z)};
+  cuuint64_t strides[2] = {256, 256ull * static_cast<cuuint64_t>(rows)};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // Packs host signs (d values of +-1) into bit words: bit i set for -1.
@@ -130,15 +145,17 @@ int num_sms() {
 }
 
 // Persistent warp-specialised kernel (d = 128): one CTA per SM.
-template <bool COUNT, bool SCALED = false>
+template <bool COUNT, bool SCALED = false, bool QK16 = false>
 int launch_v2(const void* q, const void* k, const void* v, FwdParams p, cudaStream_t stream) {
   using C = V2Config;
+  constexpr int kSmem = V2Layout<QK16>::SMEM_BYTES;
   CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, 128, p.N, p.B * p.H, 128) || !make_map(&tk, k, 128, p.N, p.B * p.Hkv, 128) ||
-      !make_map(&tv, v, 128, p.N, p.B * p.Hkv, 128))
-    return FP8ATTN_ERR_CUDA;
-  auto kern = fwd_v2_kernel<COUNT, SCALED>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+  const bool maps_ok = QK16 ? (make_map_bf16(&tq, q, p.N, p.B * p.H) && make_map_bf16(&tk, k, p.N, p.B * p.Hkv))
+                            : (make_map(&tq, q, 128, p.N, p.B * p.H, 128) &&
+                               make_map(&tk, k, 128, p.N, p.B * p.Hkv, 128));
+  if (!maps_ok || !make_map(&tv, v, 128, p.N, p.B * p.Hkv, 128)) return FP8ATTN_ERR_CUDA;
+  auto kern = fwd_v2_kernel<COUNT, SCALED, QK16>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
     return FP8ATTN_ERR_CUDA;
   // The warpgroups re-split the block's registers with setmaxnreg; that split
   // is only valid for the launch register count it was computed for.
@@ -159,7 +176,7 @@ int launch_v2(const void* q, const void* k, const void* v, FwdParams p, cudaStre
   // Scheduling groups: about two waves of units per group, capped so that the
   // K and V of the heads a group touches (and of the next group, which
   // overlaps it) stay well inside L2 (126 MB on B200).
-  const int64_t kv_head_bytes = 2ll * p.N * 128;
+  const int64_t kv_head_bytes = (QK16 ? 3ll : 2ll) * p.N * 128;
   int gh = (2 * grid + num_pairs - 1) / num_pairs;
   while (gh > 1 && ((gh + p.h_per_kv - 1) / p.h_per_kv + 1) * kv_head_bytes > (48ll << 20)) --gh;
   p.group_heads = gh < 1 ? 1 : (gh > p.B * p.H ? p.B * p.H : gh);
@@ -174,7 +191,7 @@ int launch_v2(const void* q, const void* k, const void* v, FwdParams p, cudaStre
     status = FP8ATTN_ERR_CUDA;
   } else {
     p.sched = static_cast<unsigned int*>(sched);
-    kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p, err_word);
+    kern<<<grid, C::THREADS, kSmem, stream>>>(tq, tk, tv, p, err_word);
     if (cudaGetLastError() != cudaSuccess) status = FP8ATTN_ERR_CUDA;
   }
   if (cudaFreeAsync(sched, stream) != cudaSuccess) status = FP8ATTN_ERR_CUDA;
@@ -246,7 +263,7 @@ int noalloc_setup(NoallocDevice** out) {
     auto k2 = fwd_v2_kernel<false>;
     auto k1 = fwd_v1_kernel<64, false>;
     cudaFuncAttributes attr;
-    if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, V2Config::SMEM_BYTES) !=
+    if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, V2Layout<false>::SMEM_BYTES) !=
             cudaSuccess ||
         cudaFuncGetAttributes(&attr, k2) != cudaSuccess)
       return FP8ATTN_ERR_CUDA;
@@ -284,7 +301,7 @@ int launch_v2_noalloc(const void* q, const void* k, const void* v, FwdParams p, 
   p.group_heads = gh < 1 ? 1 : (gh > p.B * p.H ? p.B * p.H : gh);
   if (cudaMemsetAsync(dev.scratch, 0, sizeof(unsigned int), stream) != cudaSuccess) return FP8ATTN_ERR_CUDA;
   p.sched = dev.scratch;
-  fwd_v2_kernel<false><<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p, dev.err_word);
+  fwd_v2_kernel<false><<<grid, C::THREADS, V2Layout<false>::SMEM_BYTES, stream>>>(tq, tk, tv, p, dev.err_word);
   return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
 }
 
@@ -346,6 +363,19 @@ extern "C" int fp8attn_fwd_scaled(const void* q, const void* k, const void* v, v
   p.k_scales = k_scales;
   p.v_scales = v_scales;
   return launch_v2<false, true>(q, k, v, p, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int fp8attn_fwd_bf16qk(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                                  int Hkv, int N, int d, int causal, float p_scale, int kv_order, void* stream) {
+  int st = validate(q, k, v, B, H, Hkv, N, d, p_scale, kv_order);
+  if (st != FP8ATTN_OK) return st;
+  if (d != 128) return FP8ATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * H * N == 0) return FP8ATTN_OK;
+  if (!o || !aligned16(o) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))) return FP8ATTN_ERR_INVALID_ARG;
+  FwdParams p = base_params(B, H, Hkv, N, causal, p_scale, kv_order);
+  p.o = o;
+  p.lse = lse;
+  return launch_v2<false, false, true>(q, k, v, p, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" int fp8attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,

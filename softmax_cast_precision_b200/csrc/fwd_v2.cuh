@@ -37,14 +37,8 @@ struct V2Config {
   static constexpr int D = 128;
   static constexpr int BM = 128;
   static constexpr int BN = 128;
-  static constexpr int STAGES = 4;              // K ring and V ring depth
+  static constexpr int STAGES = 4;              // largest ring depth (barrier arrays)
   static constexpr int TILE_BYTES = 128 * 128;  // one 128 x 128 E4M3 tile
-  static constexpr int OFF_Q = 0;                               // Q0, Q1
-  static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;          // K ring
-  static constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;     // V ring
-  static constexpr int OFF_P = OFF_V + STAGES * TILE_BYTES;     // P0 x2, P1 x2 (double-buffered)
-  static constexpr int OFF_BAR = OFF_P + 4 * TILE_BYTES;
-  static constexpr int SMEM_BYTES = OFF_BAR + 320 + 1024;  // control block + alignment slack
   static constexpr int THREADS = 384;  // 3 warpgroups
   // Register split (setmaxnreg): the block launches with 168 registers per
   // thread (65536 / 384 rounded down to a multiple of 8); the producer
@@ -53,6 +47,22 @@ struct V2Config {
   static constexpr int SOFTMAX_REGS = 208;
   static constexpr int PRODUCER_REGS = 80;
   static constexpr uint32_t TMEM_COLS = 512;
+};
+
+// Shared-memory layout.  QK16 = false: Q and K are E4M3 (16 KB tiles, one
+// 128-byte swizzle panel), K and V rings of 4 stages.  QK16 = true: Q and K
+// are bfloat16 (32 KB tiles: two 64-column panels of 128-byte rows), rings
+// of 2 stages; V and P^ stay E4M3 either way.
+template <bool QK16>
+struct V2Layout {
+  static constexpr int STAGES = QK16 ? 2 : 4;
+  static constexpr int QK_TILE = QK16 ? 2 * V2Config::TILE_BYTES : V2Config::TILE_BYTES;
+  static constexpr int OFF_Q = 0;                                         // Q0, Q1
+  static constexpr int OFF_K = OFF_Q + 2 * QK_TILE;                       // K ring
+  static constexpr int OFF_V = OFF_K + STAGES * QK_TILE;                  // V ring
+  static constexpr int OFF_P = OFF_V + STAGES * V2Config::TILE_BYTES;     // P0 x2, P1 x2 (double-buffered)
+  static constexpr int OFF_BAR = OFF_P + 4 * V2Config::TILE_BYTES;
+  static constexpr int SMEM_BYTES = OFF_BAR + 320 + 1024;  // control block + alignment slack
 };
 
 // Shared-memory control block.
@@ -72,7 +82,8 @@ struct V2Bars {
   uint32_t tmem_base;
   volatile uint32_t abort;
 };
-static_assert(V2Config::SMEM_BYTES <= 232448, "exceeds the 227 KB shared-memory limit per block");
+static_assert(V2Layout<false>::SMEM_BYTES <= 232448 && V2Layout<true>::SMEM_BYTES <= 232448,
+              "exceeds the 227 KB shared-memory limit per block");
 static_assert(sizeof(V2Bars) <= 320, "control block exceeds its shared-memory slot");
 static_assert(2 * 128 * V2Config::SOFTMAX_REGS + 128 * V2Config::PRODUCER_REGS <=
                   V2Config::THREADS * V2Config::LAUNCH_REGS,
@@ -162,14 +173,17 @@ constexpr int kPolyPairs = 2;
 // SCALED: the inputs carry descales (FwdParams q/k/v_scales) and optionally
 // a rotation to undo on the output; the running maximum is then kept in
 // log2 units of the descaled logits, whose scale changes from tile to tile.
-template <bool COUNT, bool SCALED = false>
+// QK16: Q and K are bfloat16 and S = Q K^T runs as a kind::f16 product (the
+// P-cast and P V are unchanged).
+template <bool COUNT, bool SCALED = false, bool QK16 = false>
 __global__ void __launch_bounds__(V2Config::THREADS, 1)
     fwd_v2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p, uint32_t* err_word) {
   using C = V2Config;
+  using L = V2Layout<QK16>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  V2Bars* bars = reinterpret_cast<V2Bars*>(base + C::OFF_BAR);
+  V2Bars* bars = reinterpret_cast<V2Bars*>(base + L::OFF_BAR);
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
@@ -191,7 +205,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
     mbar_init(&bars->q_full[0], 1);
     mbar_init(&bars->q_full[1], 1);
     mbar_init(&bars->q_free, 256);
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < L::STAGES; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->k_free[s], 256);
@@ -247,32 +261,36 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         const UnitGeom g = unit_geom(p, u);
         if (q_it > 0) ok = v2_wait(bars, &bars->q_free, (q_it - 1) & 1, err_word, kErrTimeoutPipe);
         if (!ok) break;
-        mbar_arrive_expect_tx(&bars->q_full[0], C::TILE_BYTES);
-        tma_load_3d(base + C::OFF_Q, &tm_q, &bars->q_full[0], 0, g.q0, g.zq);
+        // A Q or K tile is one box, or for bfloat16 two boxes of 64 columns
+        // (one 128-byte swizzle panel each, 16 KB apart).
+        auto load_qk = [&](uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row, int slab) {
+          mbar_arrive_expect_tx(bar, L::QK_TILE);
+          tma_load_3d(dst, map, bar, 0, row, slab);
+          if constexpr (QK16) tma_load_3d(dst + C::TILE_BYTES, map, bar, 64, row, slab);
+        };
+        load_qk(base + L::OFF_Q, &tm_q, &bars->q_full[0], g.q0, g.zq);
         ++q_done[0];
         if (g.last[1] >= 0) {
-          mbar_arrive_expect_tx(&bars->q_full[1], C::TILE_BYTES);
-          tma_load_3d(base + C::OFF_Q + C::TILE_BYTES, &tm_q, &bars->q_full[1], 0, g.q0 + 128, g.zq);
+          load_qk(base + L::OFF_Q + L::QK_TILE, &tm_q, &bars->q_full[1], g.q0 + 128, g.zq);
           ++q_done[1];
         }
         ++q_it;
         for (int idx = 0; idx < g.ntiles; ++idx) {
           const int t = stream_tile(p, g, idx);
-          const int st = kv_it % C::STAGES;
+          const int st = kv_it % L::STAGES;
           // K is released once both query tiles have read their S for it, V
           // once both have seen its P V products complete.
-          if (kv_it >= C::STAGES) {
-            ok = v2_wait(bars, &bars->k_free[st], ((kv_it / C::STAGES) - 1) & 1, err_word, kErrTimeoutPipe);
+          if (kv_it >= L::STAGES) {
+            ok = v2_wait(bars, &bars->k_free[st], ((kv_it / L::STAGES) - 1) & 1, err_word, kErrTimeoutPipe);
             if (!ok) break;
           }
-          mbar_arrive_expect_tx(&bars->k_full[st], C::TILE_BYTES);
-          tma_load_3d(base + C::OFF_K + st * C::TILE_BYTES, &tm_k, &bars->k_full[st], 0, t * 128, g.zkv);
-          if (kv_it >= C::STAGES) {
-            ok = v2_wait(bars, &bars->v_free[st], ((kv_it / C::STAGES) - 1) & 1, err_word, kErrTimeoutPipe);
+          load_qk(base + L::OFF_K + st * L::QK_TILE, &tm_k, &bars->k_full[st], t * 128, g.zkv);
+          if (kv_it >= L::STAGES) {
+            ok = v2_wait(bars, &bars->v_free[st], ((kv_it / L::STAGES) - 1) & 1, err_word, kErrTimeoutPipe);
             if (!ok) break;
           }
           mbar_arrive_expect_tx(&bars->v_full[st], C::TILE_BYTES);
-          tma_load_3d(base + C::OFF_V + st * C::TILE_BYTES, &tm_v, &bars->v_full[st], 0, t * 128, g.zkv);
+          tma_load_3d(base + L::OFF_V + st * C::TILE_BYTES, &tm_v, &bars->v_full[st], 0, t * 128, g.zkv);
           ++kv_it;
         }
       }
@@ -281,9 +299,9 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         // released: the last Q pair and the last STAGES K/V tiles.
         if (q_done[0] > 0) drain_wait(&bars->q_full[0], (q_done[0] - 1) & 1);
         if (q_done[1] > 0) drain_wait(&bars->q_full[1], (q_done[1] - 1) & 1);
-        for (uint32_t i = (kv_it > C::STAGES ? kv_it - C::STAGES : 0); i < kv_it; ++i) {
-          drain_wait(&bars->k_full[i % C::STAGES], (i / C::STAGES) & 1);
-          drain_wait(&bars->v_full[i % C::STAGES], (i / C::STAGES) & 1);
+        for (uint32_t i = (kv_it > L::STAGES ? kv_it - L::STAGES : 0); i < kv_it; ++i) {
+          drain_wait(&bars->k_full[i % L::STAGES], (i / L::STAGES) & 1);
+          drain_wait(&bars->v_full[i % L::STAGES], (i / L::STAGES) & 1);
         }
       }
     }
@@ -302,16 +320,17 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
     // while this form (and an unrolled single-warp form) is exact.
     auto mma_role = [&](auto kc) {
     constexpr int k = decltype(kc)::value;
-    constexpr uint32_t idesc_qk = idesc_e4m3_f32(128, 128, false, false);
+    constexpr uint32_t idesc_qk = QK16 ? idesc_bf16_f32(128, 128) : idesc_e4m3_f32(128, 128, false, false);
     constexpr uint32_t idesc_pv = idesc_e4m3_f32(128, 128, false, true);
     // Descriptors are built once: a K step of 32 keys/columns moves the
     // start-address field (bytes >> 4) by 2 for the K-major operands (32
     // bytes along the row) and by 256 for V (32 rows of 128 bytes).
-    constexpr uint64_t kTile = C::TILE_BYTES >> 4;  // one 16 KB tile in the address field
-    const uint64_t dQ = smem_desc(smem_u32(base + C::OFF_Q), 16, 1024, 2) + k * kTile;
-    const uint64_t dK0 = smem_desc(smem_u32(base + C::OFF_K), 16, 1024, 2);
-    const uint64_t dV0 = smem_desc(smem_u32(base + C::OFF_V), 128 * 128, 1024, 2);
-    const uint64_t dP = smem_desc(smem_u32(base + C::OFF_P), 16, 1024, 2) + 2 * k * kTile;
+    constexpr uint64_t kTile = C::TILE_BYTES >> 4;  // one 16 KB tile (or panel) in the address field
+    constexpr uint64_t kQKTile = L::QK_TILE >> 4;
+    const uint64_t dQ = smem_desc(smem_u32(base + L::OFF_Q), 16, 1024, 2) + k * kQKTile;
+    const uint64_t dK0 = smem_desc(smem_u32(base + L::OFF_K), 16, 1024, 2);
+    const uint64_t dV0 = smem_desc(smem_u32(base + L::OFF_V), 128 * 128, 1024, 2);
+    const uint64_t dP = smem_desc(smem_u32(base + L::OFF_P), 16, 1024, 2) + 2 * k * kTile;
     const uint32_t tS = tmem + 128 * k;
     const uint32_t tO = tmem + 256 + 128 * k;
     uint32_t kv_base = 0, q_it = 0, s_cnt = 0, p_cnt = 0, units = 0;
@@ -335,15 +354,25 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         if (idx < lo + nk) {
           // S_k = Q_k K^T once K has landed and softmax k has read its previous S.
           const uint32_t it = unit_base + idx;
-          const int st = it % C::STAGES;
-          ok = wait_all(&bars->k_full[st], (it / C::STAGES) & 1, kErrTimeoutKV);
+          const int st = it % L::STAGES;
+          ok = wait_all(&bars->k_full[st], (it / L::STAGES) & 1, kErrTimeoutKV);
           if (ok && s_cnt > 0) ok = wait_all(&bars->s_free[k], (s_cnt - 1) & 1, kErrTimeoutPipe);
           if (!ok) break;
           tc_fence_after();
           if (lane == 0) {
-            const uint64_t db = dK0 + st * kTile;
+            const uint64_t db = dK0 + st * kQKTile;
+            if constexpr (QK16) {
+              // K = 16 per instruction: 32 bytes along the row (+2), four
+              // steps per 128-byte panel, then the next panel (+16 KB).
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tS, dQ + 2 * kk, db + 2 * kk, idesc_qk, kk > 0);
+              for (int kk = 0; kk < 8; ++kk) {
+                const uint64_t off = (kk >> 2) * kTile + 2 * (kk & 3);
+                mma_bf16_ss(tS, dQ + off, db + off, idesc_qk, kk > 0);
+              }
+            } else {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tS, dQ + 2 * kk, db + 2 * kk, idesc_qk, kk > 0);
+            }
             mma_commit(&bars->s_full[k]);
           }
           __syncwarp();
@@ -353,10 +382,10 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
           // O_k += P^_k V for the previous tile once softmax k has written P^_k
           // (and, at a unit's first tile, has read out the previous unit's O_k).
           const uint32_t it = unit_base + idx - 1;
-          const int st = it % C::STAGES;
+          const int st = it % L::STAGES;
           const bool first = (idx - 1 == lo);
           ok = wait_all(&bars->p_full[k], p_cnt & 1, kErrTimeoutPipe);
-          if (ok) ok = wait_all(&bars->v_full[st], (it / C::STAGES) & 1, kErrTimeoutKV);
+          if (ok) ok = wait_all(&bars->v_full[st], (it / L::STAGES) & 1, kErrTimeoutKV);
           if (ok && first && units > 0) ok = wait_all(&bars->o_free[k], (units - 1) & 1, kErrTimeoutPipe);
           if (!ok) break;
           tc_fence_after();
@@ -393,7 +422,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tS = tmem + 128 * k + lane_off;
     const uint32_t tO = tmem + 256 + 128 * k + lane_off;
-    const uint32_t sPk = smem_u32(base + C::OFF_P + 2 * k * C::TILE_BYTES);
+    const uint32_t sPk = smem_u32(base + L::OFF_P + 2 * k * C::TILE_BYTES);
     uint32_t s_it = 0, o_it = 0, p_cnt = 0;
     uint32_t kv_base = 0;  // stream position of the unit's first KV tile (ring stage bookkeeping)
     bool ok = true;
@@ -472,7 +501,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         // This S has completed, so the K stage it read (and, at the unit's
         // last tile, the Q pair) may be refilled once the other query tile is
         // done with them too; a tile it does not use counts twice here.
-        const int stage = static_cast<int>((unit_base + idx) % C::STAGES);
+        const int stage = static_cast<int>((unit_base + idx) % L::STAGES);
         const uint32_t cnt = (t <= last_other) ? 1u : 2u;
         mbar_arrive_cnt(&bars->k_free[stage], cnt);
         if (p.reverse ? (t == 0) : (t == last)) mbar_arrive_cnt(&bars->q_free, last_other >= 0 ? 1u : 2u);

@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.fp8attn_quantize.restype = i32
         L.fp8attn_fwd_scaled.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, P]
         L.fp8attn_fwd_scaled.restype = i32
+        L.fp8attn_fwd_bf16qk.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, P]
+        L.fp8attn_fwd_bf16qk.restype = i32
         L.fp8attn_pzero_count.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, P]
         L.fp8attn_pzero_count.restype = i32
         L.fp8attn_kv_tile.argtypes = [i32]
@@ -180,6 +182,26 @@ def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Te
                                    _stream_ptr(q.device, stream))
     if st != OK:
         raise Fp8AttnError(st, "fp8attn_fwd_noalloc")
+
+
+def fwd_bf16qk(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_scale: float = 256.0,
+               kv_order="reverse", with_lse: bool = True, stream=None):
+    """Forward pass with bfloat16 q [B,H,N,128], k [B,Hkv,N,128] and E4M3 v [B,Hkv,N,128] (device
+    tensors): S = Q K^T on the 16-bit tensor-core path, then the same P-cast and P V as ``fwd``."""
+    if q.dtype != torch.bfloat16 or k.dtype != torch.bfloat16:
+        raise TypeError("q and k must be bfloat16")
+    v = _bytes(v)
+    q, k = q.contiguous(), k.contiguous()
+    B, H, Hkv, N, d = _shapes(q, k, v)
+    if not q.is_cuda:
+        raise ValueError("fwd_bf16qk takes device tensors")
+    o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if with_lse else None
+    st = lib().fp8attn_fwd_bf16qk(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, N, d, int(bool(causal)),
+                                  ctypes.c_float(p_scale), _order(kv_order), _stream_ptr(q.device, stream))
+    if st != OK:
+        raise Fp8AttnError(st, "fp8attn_fwd_bf16qk")
+    return o, lse
 
 
 def _host_signs(signs, d: int):

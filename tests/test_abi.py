@@ -31,6 +31,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ["fp8attn_fwd", "fp8attn_fwd_noalloc", "fp8attn_fwd_scaled", "fp8attn_quantize",
+                     "fp8attn_fwd_bf16qk",
                      "fp8attn_pzero_count", "fp8attn_kv_tile", "fp8attn_status_str",
                      "fp8attn_check_error"]:
         assert required in names
@@ -74,7 +75,7 @@ def _call_fwd(fp8, q=16, k=16, v=16, o=16, B=1, H=2, Hkv=1, N=128, d=128, causal
     (dict(S=float("nan")), 1), (dict(S=2.0**65), 1), (dict(S=2.0**-65), 1), (dict(order=2), 1), (dict(q=0), 1), (dict(k=8), 1), (dict(v=4), 1),
     (dict(o=0), 1), (dict(o=24), 1), (dict(B=70000), 2),
 ])
-@pytest.mark.parametrize("entry", ["fp8attn_fwd", "fp8attn_fwd_noalloc"])
+@pytest.mark.parametrize("entry", ["fp8attn_fwd", "fp8attn_fwd_noalloc", "fp8attn_fwd_bf16qk"])
 def test_invalid_arguments_rejected_without_launch(fp8, kw, expected, entry):
     assert _call_fwd(fp8, entry=entry, **kw) == expected
 
@@ -156,3 +157,7 @@ def _call_fwd_scaled(fp8, qs=16, ks=16, vs=16, d=128, signs=None, N=128, S=256.0
 ])
 def test_fwd_scaled_validation(fp8, kw, expected):
     assert _call_fwd_scaled(fp8, **kw) == expected
+
+
+def test_bf16qk_is_d128_only(fp8):
+    assert _call_fwd(fp8, d=64, entry="fp8attn_fwd_bf16qk") == fp8.ERR_UNSUPPORTED
