@@ -14,6 +14,9 @@ host cores instead, on a bounded sample of the same workload per step.
 --path wide starts from bfloat16 Q, K, V instead: one step quantises them
 (random-sign Hadamard rotation, Q and K per 128-row block, V per head) and
 runs the scaled forward pass, which rotates the output back.
+
+--path bf16qk keeps Q and K in bfloat16 (S = Q K^T on the 16-bit tensor-core
+path) with E4M3 V: the P-cast summary's kernel-faithful setting.
 """
 from __future__ import annotations
 
@@ -58,8 +61,9 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--path", default="fp8", choices=["fp8", "wide"],
-                    help="fp8: E4M3 inputs (the headline); wide: bfloat16 inputs quantised in the step")
+    ap.add_argument("--path", default="fp8", choices=["fp8", "wide", "bf16qk"],
+                    help="fp8: E4M3 inputs (the headline); wide: bfloat16 inputs quantised in the step; "
+                         "bf16qk: bfloat16 Q and K, E4M3 V")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (used under ncu)")
     return ap.parse_args()
@@ -403,6 +407,130 @@ def run_wide(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+BF16QK_WORKLOAD_DESC = ("prefill32k with bfloat16 Q and K: B=1 H=32 N=32768 d=128 causal, Delta=7 sink (k=4), "
+                        "E4M3 V, S=256, reverse KV order")
+
+
+def run_bf16qk(args, rank, world, local_rank):
+    """bfloat16 Q and K, E4M3 V: one fp8attn_fwd_bf16qk launch per step."""
+    import torch
+
+    from softmax_cast_precision_b200 import fp8attn
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    w = WORKLOAD
+    q, k, v, _ = wide_inputs(rank_seed(rank))
+    v8 = torch.from_numpy(np.clip(v, -448, 448)).to(torch.float8_e4m3fn).view(torch.uint8)
+    qb, kb = (torch.from_numpy(x).to(device).to(torch.bfloat16) for x in (q, k))
+    vd = v8.to(device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        return fp8attn.fwd_bf16qk(qb, kb, vd, causal=w.causal, p_scale=P_SCALE, kv_order=KV_ORDER, stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    fp8attn.check_error(stream=stream, device=device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize(device)
+        ev[0].record(stream)
+        for i in range(args.steps):
+            o, lse = step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+    fp8attn.check_error(stream=stream, device=device)
+    per_step = [ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps)]
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), dist, device)
+    ms_per_step = total_ms / args.steps
+    flops = w.flops()
+    # End to end from pinned host buffers.
+    qh, kh, vh = qb.cpu().pin_memory(), kb.cpu().pin_memory(), v8.pin_memory()
+    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    qd, kd, vd2 = torch.empty_like(qb), torch.empty_like(kb), torch.empty_like(vd)
+
+    def e2e_step():
+        for dst, src in ((qd, qh), (kd, kh), (vd2, vh)):
+            dst.copy_(src, non_blocking=True)
+        oo, ll = fp8attn.fwd_bf16qk(qd, kd, vd2, causal=w.causal, p_scale=P_SCALE, kv_order=KV_ORDER, stream=stream)
+        oh.copy_(oo, non_blocking=True)
+        lh.copy_(ll, non_blocking=True)
+
+    e2e_step()
+    e2e_steps = max(3, min(args.steps, 10))
+    barrier()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, device)
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+    mse = None
+    if rank == 0:
+        mse = wide_mse_vs_fp64(qb, kb, vd.view(torch.float8_e4m3fn).float(), o, sample_rows(w.N, 256))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peak_bf16, _, peak_src = fp8_peak()
+    peak_bf16 /= FP8_OVER_BF16
+    # Half of the FLOPs (Q K^T) at the 16-bit rate, half (P V) at the FP8 rate.
+    peak_mix = 1.0 / (0.5 / peak_bf16 + 0.5 / (peak_bf16 * FP8_OVER_BF16))
+    kernel_ms = statistics.mean(per_step)
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": aggregate_throughput(flops, world, ms_per_step), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 QK / e4m3 PV", "data": "synthetic",
+        "config": {"workload": BF16QK_WORKLOAD_DESC, "flop_per_step_per_gpu": flops,
+                   "l2": "inputs exceed L2 (671 MB)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_mix, "unit": "TFLOP/s",
+                     "frac": achieved / peak_mix, "traffic": None,
+                     "peak_source": f"{peak_src}: half the FLOPs at the bf16 cuBLAS burst rate, half at x "
+                                    f"{FP8_OVER_BF16} (FP8/BF16 nominal)"},
+        "e2e": {"value": aggregate_throughput(flops, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "clocks": clk.summary(),
+        "mse_vs_fp64": {"value": mse, "rows": "256 evenly spaced query rows of each head",
+                        "reference": "PyTorch float64 softmax(QK^T/sqrt(d))V on the bfloat16 Q, K and decoded V"},
+    }
+    if not args.skip_cpu_baseline:
+        import oracle
+
+        rows = sample_rows(w.N, CPU_SAMPLE_ROWS)
+        t0 = time.perf_counter()
+        oracle.emulate(q, k, v8.numpy(), causal=w.causal, block_n=128, p_scale=P_SCALE, reverse=bool(KV_ORDER),
+                       rows=rows)
+        dt = time.perf_counter() - t0
+        f = 4.0 * w.d * visible_pairs(rows, w.N, w.causal) * w.B * w.H
+        line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                                "sample": f"blockwise emulator on {len(rows)} evenly spaced query rows of each head "
+                                          f"({f / 1e12:.3f} TFLOP in {dt:.1f} s)"}
+    print(json.dumps(line), flush=True)
+
+
 def hbm_peak() -> float:
     try:
         with open(PEAKS_FILE) as fh:
@@ -494,9 +622,13 @@ def main():
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
+        if args.path == "bf16qk":
+            raise SystemExit("--impl reference covers --path fp8 and wide")
         return run_reference_wide(args, rank) if args.path == "wide" else run_reference(args, rank, world)
     if args.path == "wide":
         return run_wide(args, rank, world, local_rank)
+    if args.path == "bf16qk":
+        return run_bf16qk(args, rank, world, local_rank)
 
     import torch
 
