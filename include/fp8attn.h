@@ -152,6 +152,29 @@ int fp8attn_fwd_bf16qk(const void* q, const void* k, const void* v, void* o, flo
                        float p_scale, int kv_order, void* stream);
 
 /*
+ * Decode / split-KV forward pass: one query row per (batch, head) against
+ * all N keys, q [B, H, d] E4M3, k and v [B, Hkv, N, d] E4M3 (device), o
+ * [B, H, d] bfloat16, lse [B, H] float32 (may be NULL).  The keys are cut
+ * into splits of split_tiles consecutive 128-key tiles; each split runs the
+ * blockwise online softmax with the P-cast on its own, its tiles walked in
+ * kv_order, and the splits are merged exactly through their maxima and
+ * sums ("Attenzione flash e domanda sulla lunghezza della sequenza", section
+ * "La ricorrenza softmax online"; "P-Cast Precision in FP8 Attention",
+ * technical summary, section 1).  No causal mask (the query is the last
+ * position).  workspace is caller-owned device memory of at least
+ * fp8attn_decode_workspace_bytes(B, H, N, split_tiles) bytes, 16-byte
+ * aligned, overwritten by the call.  d must be 128 and H / Hkv at most 8
+ * (FP8ATTN_ERR_UNSUPPORTED otherwise); N >= 1; k, v, o 16-byte aligned.
+ */
+int fp8attn_decode(const void* q, const void* k, const void* v, void* o, float* lse,
+                   void* workspace, unsigned long long workspace_bytes,
+                   int B, int H, int Hkv, int N, int d, float p_scale, int kv_order,
+                   int split_tiles, void* stream);
+
+/* Workspace bytes fp8attn_decode needs (0 for invalid sizes). */
+unsigned long long fp8attn_decode_workspace_bytes(int B, int H, int N, int split_tiles);
+
+/*
  * Allocation-free forward pass.  The pages have no counterpart of this call:
  * it is an interface for callers that cannot let the library allocate device
  * memory -- programs that hand the whole device memory to their own allocator

@@ -16,6 +16,7 @@
 #include "fwd_v1.cuh"
 #include "fwd_v2.cuh"
 #include "quantize.cuh"
+#include "decode.cuh"
 
 namespace fp8attn {
 
@@ -449,6 +450,57 @@ extern "C" int fp8attn_quantize(const void* x, int x_dtype, void* xq, float* sca
   p.x_f32 = x_dtype;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 128 ? launch_quantize<32>(p, s) : launch_quantize<16>(p, s);
+}
+
+extern "C" unsigned long long fp8attn_decode_workspace_bytes(int B, int H, int N, int split_tiles) {
+  if (B <= 0 || H <= 0 || N <= 0 || split_tiles <= 0) return 0;
+  const int64_t ntiles = (static_cast<int64_t>(N) + 127) / 128;
+  const int64_t splits = (ntiles + split_tiles - 1) / split_tiles;
+  return static_cast<unsigned long long>(B) * H * splits * fp8attn::kDecodePartStride * sizeof(float);
+}
+
+extern "C" int fp8attn_decode(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,
+                              unsigned long long workspace_bytes, int B, int H, int Hkv, int N, int d,
+                              float p_scale, int kv_order, int split_tiles, void* stream) {
+  using namespace fp8attn;
+  if (B < 0 || N < 0 || H < 1 || Hkv < 1 || H % Hkv != 0 || split_tiles < 1) return FP8ATTN_ERR_INVALID_ARG;
+  if (d != 128 || H / Hkv > kDecodeMaxG) return FP8ATTN_ERR_UNSUPPORTED;
+  if (!(p_scale >= 0x1p-64f) || !(p_scale <= 0x1p64f)) return FP8ATTN_ERR_INVALID_ARG;
+  if (kv_order != 0 && kv_order != 1) return FP8ATTN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B) * Hkv > 65535 || static_cast<int64_t>(B) * H > 0x7fffffff)
+    return FP8ATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * H == 0) return FP8ATTN_OK;
+  if (N == 0) return FP8ATTN_ERR_INVALID_ARG;  // a query with no key has no softmax
+  if (!q || !k || !v || !o || !workspace || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      !aligned16(workspace) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FP8ATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < fp8attn_decode_workspace_bytes(B, H, N, split_tiles)) return FP8ATTN_ERR_INVALID_ARG;
+  DecodeParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.q = static_cast<const uint8_t*>(q);
+  p.k = static_cast<const uint8_t*>(k);
+  p.v = static_cast<const uint8_t*>(v);
+  p.part = static_cast<float*>(workspace);
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.G = H / Hkv;
+  p.ntiles = (N + 127) / 128;
+  p.split_tiles = split_tiles;
+  p.splits = (p.ntiles + split_tiles - 1) / split_tiles;
+  p.reverse = kv_order;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
+  p.log2_p_scale = static_cast<float>(std::log2(static_cast<double>(p_scale)));
+  constexpr int kSmem = 4 * 128 * 128 + 2 * kDecodeMaxG * 128 * 4 + 4 * kDecodeMaxG * 4;
+  if (cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
+    return FP8ATTN_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  decode_split_kernel<<<dim3(p.splits, B * Hkv), 128, kSmem, s>>>(p);
+  decode_combine_kernel<<<B * H, 128, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
 }
 
 extern "C" int fp8attn_kv_tile(int d) {

@@ -58,6 +58,11 @@ def lib() -> ctypes.CDLL:
         L.fp8attn_fwd_scaled.restype = i32
         L.fp8attn_fwd_bf16qk.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, P]
         L.fp8attn_fwd_bf16qk.restype = i32
+        u64 = ctypes.c_ulonglong
+        L.fp8attn_decode.argtypes = [P, P, P, P, P, P, u64, i32, i32, i32, i32, i32, f32, i32, i32, P]
+        L.fp8attn_decode.restype = i32
+        L.fp8attn_decode_workspace_bytes.argtypes = [i32, i32, i32, i32]
+        L.fp8attn_decode_workspace_bytes.restype = u64
         L.fp8attn_pzero_count.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, P]
         L.fp8attn_pzero_count.restype = i32
         L.fp8attn_kv_tile.argtypes = [i32]
@@ -201,6 +206,32 @@ def fwd_bf16qk(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: boo
                                   ctypes.c_float(p_scale), _order(kv_order), _stream_ptr(q.device, stream))
     if st != OK:
         raise Fp8AttnError(st, "fp8attn_fwd_bf16qk")
+    return o, lse
+
+
+def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, p_scale: float = 256.0, kv_order="reverse",
+           split_tiles: int = 16, with_lse: bool = True, workspace: torch.Tensor | None = None, stream=None):
+    """Decode step: q [B,H,d] (one query row per head) against k, v [B,Hkv,N,d], all E4M3 on the GPU.
+
+    The keys are processed in splits of ``split_tiles`` 128-key tiles that are
+    merged exactly; returns (o [B,H,d] bfloat16, lse [B,H] or None).
+    """
+    q, k, v = _bytes(q), _bytes(k), _bytes(v)
+    if q.dim() != 3 or k.dim() != 4 or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("q must be [B,H,d]; k and v [B,Hkv,N,d]")
+    B, H, d = (int(x) for x in q.shape)
+    Hkv, N = int(k.shape[1]), int(k.shape[2])
+    if not q.is_cuda:
+        raise ValueError("decode takes device tensors")
+    need = int(lib().fp8attn_decode_workspace_bytes(B, H, N, int(split_tiles)))
+    ws = workspace if workspace is not None else torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    o = torch.empty((B, H, d), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if with_lse else None
+    st = lib().fp8attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(),
+                              B, H, Hkv, N, d, ctypes.c_float(p_scale), _order(kv_order), int(split_tiles),
+                              _stream_ptr(q.device, stream))
+    if st != OK:
+        raise Fp8AttnError(st, "fp8attn_decode")
     return o, lse
 
 

@@ -31,7 +31,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ["fp8attn_fwd", "fp8attn_fwd_noalloc", "fp8attn_fwd_scaled", "fp8attn_quantize",
-                     "fp8attn_fwd_bf16qk",
+                     "fp8attn_fwd_bf16qk", "fp8attn_decode", "fp8attn_decode_workspace_bytes",
                      "fp8attn_pzero_count", "fp8attn_kv_tile", "fp8attn_status_str",
                      "fp8attn_check_error"]:
         assert required in names
@@ -161,3 +161,26 @@ def test_fwd_scaled_validation(fp8, kw, expected):
 
 def test_bf16qk_is_d128_only(fp8):
     assert _call_fwd(fp8, d=64, entry="fp8attn_fwd_bf16qk") == fp8.ERR_UNSUPPORTED
+
+
+def test_decode_workspace_and_validation(fp8):
+    L = fp8.lib()
+    assert L.fp8attn_decode_workspace_bytes(2, 8, 1000, 3) == 2 * 8 * 3 * 130 * 4  # 8 tiles -> 3 splits
+    assert L.fp8attn_decode_workspace_bytes(0, 8, 1000, 3) == 0
+    assert L.fp8attn_decode_workspace_bytes(1, 8, 1000, 0) == 0
+    P = ctypes.c_void_p
+
+    def call(d=128, H=8, Hkv=2, N=1000, split=3, ws=16, wsb=10 ** 6, S=256.0, order=1, B=1):
+        return L.fp8attn_decode(P(16), P(16), P(16), P(16), P(0), P(ws), wsb, B, H, Hkv, N, d, ctypes.c_float(S),
+                                order, split, P(0))
+    assert call(d=64) == fp8.ERR_UNSUPPORTED
+    assert call(H=32, Hkv=2) == fp8.ERR_UNSUPPORTED  # 16 query heads per kv head
+    assert call(H=6, Hkv=4) == fp8.ERR_INVALID_ARG
+    assert call(split=0) == fp8.ERR_INVALID_ARG
+    assert call(wsb=100) == fp8.ERR_INVALID_ARG
+    assert call(ws=0) == fp8.ERR_INVALID_ARG
+    assert call(ws=8) == fp8.ERR_INVALID_ARG
+    assert call(N=0) == fp8.ERR_INVALID_ARG
+    assert call(S=0.0) == fp8.ERR_INVALID_ARG
+    assert call(order=3) == fp8.ERR_INVALID_ARG
+    assert call(B=0) == fp8.OK
