@@ -17,6 +17,9 @@ runs the scaled forward pass, which rotates the output back.
 
 --path bf16qk keeps Q and K in bfloat16 (S = Q K^T on the 16-bit tensor-core
 path) with E4M3 V: the P-cast summary's kernel-faithful setting.
+
+--path decode times the split-KV decode pass (B=32, H=32, Hkv=8, N=32768,
+one query row per head, 16-tile splits) against the HBM roofline.
 """
 from __future__ import annotations
 
@@ -61,9 +64,9 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--path", default="fp8", choices=["fp8", "wide", "bf16qk"],
+    ap.add_argument("--path", default="fp8", choices=["fp8", "wide", "bf16qk", "decode"],
                     help="fp8: E4M3 inputs (the headline); wide: bfloat16 inputs quantised in the step; "
-                         "bf16qk: bfloat16 Q and K, E4M3 V")
+                         "bf16qk: bfloat16 Q and K, E4M3 V; decode: one query row per head, split-KV")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (used under ncu)")
     return ap.parse_args()
@@ -531,6 +534,116 @@ def run_bf16qk(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+DECODE_SHAPE = dict(B=32, H=32, Hkv=8, N=32768, split_tiles=16)
+DECODE_METRIC = "FP8 split-KV decode GB/s of K/V read (HBM roofline)"
+
+
+def run_decode(args, rank, world, local_rank):
+    """One fp8attn_decode call per step (split pass + merge), timed with CUDA events."""
+    import torch
+
+    from softmax_cast_precision_b200 import fp8attn
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    sh = DECODE_SHAPE
+    B, H, Hkv, N, split = sh["B"], sh["H"], sh["Hkv"], sh["N"], sh["split_tiles"]
+    g = torch.Generator(device=device).manual_seed(rank_seed(rank))
+
+    def mk(*shape):
+        return torch.randn(shape, device=device, generator=g).clamp(-448, 448).to(torch.float8_e4m3fn).view(
+            torch.uint8)
+
+    q, k, v = mk(B, H, 128), mk(B, Hkv, N, 128), mk(B, Hkv, N, 128)
+    ws = torch.empty(int(fp8attn.lib().fp8attn_decode_workspace_bytes(B, H, N, split)), dtype=torch.uint8,
+                     device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        return fp8attn.decode(q, k, v, p_scale=P_SCALE, kv_order=KV_ORDER, split_tiles=split, workspace=ws,
+                              stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    fp8attn.check_error(stream=stream, device=device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize(device)
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+    fp8attn.check_error(stream=stream, device=device)
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), dist, device)
+    ms_per_step = total_ms / args.steps
+    kv_bytes = 2 * k.numel()
+    alg_bytes = kv_bytes + q.numel() + B * H * 128 * 2 + B * H * 4
+    # End to end: K/V from pinned host memory (the cache would normally stay resident; this is the
+    # worst case the public call can be timed at).
+    qh, kh, vh = q.cpu().pin_memory(), k.cpu().pin_memory(), v.cpu().pin_memory()
+    qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    oh = torch.empty((B, H, 128), dtype=torch.bfloat16, pin_memory=True)
+    lh = torch.empty((B, H), dtype=torch.float32, pin_memory=True)
+
+    def e2e_step():
+        for dst, src in ((qd, qh), (kd, kh), (vd, vh)):
+            dst.copy_(src, non_blocking=True)
+        o, lse = fp8attn.decode(qd, kd, vd, p_scale=P_SCALE, kv_order=KV_ORDER, split_tiles=split, workspace=ws,
+                                stream=stream)
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(3):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / 3, dist, device)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    kernel_ms = statistics.mean(ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps))
+    hbm = hbm_peak()
+    achieved = alg_bytes / (kernel_ms * 1e-3) / 1e9
+    line = {
+        "metric": DECODE_METRIC, "value": kv_bytes * world / (ms_per_step * 1e-3) / 1e9, "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": f"decode: B={B} H={H} Hkv={Hkv} N={N} d=128, one query row per head, E4M3 Q/K/V "
+                               f"N(0,1), S=256, reverse order inside {split}-tile splits",
+                   "l2": f"K/V exceed L2 ({kv_bytes / 1e9:.2f} GB)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "gpu_launches": 2 * args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": None, "algorithmic_bytes": alg_bytes,
+                     "peak_source": "measured copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"},
+        "e2e": {"value": kv_bytes * world / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": q.numel() + 2 * k.numel(), "d2h_bytes_per_step": B * H * (128 * 2 + 4),
+                "ms_per_step": e2e_ms},
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+
+
 def hbm_peak() -> float:
     try:
         with open(PEAKS_FILE) as fh:
@@ -622,13 +735,15 @@ def main():
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
-        if args.path == "bf16qk":
+        if args.path in ("bf16qk", "decode"):
             raise SystemExit("--impl reference covers --path fp8 and wide")
         return run_reference_wide(args, rank) if args.path == "wide" else run_reference(args, rank, world)
     if args.path == "wide":
         return run_wide(args, rank, world, local_rank)
     if args.path == "bf16qk":
         return run_bf16qk(args, rank, world, local_rank)
+    if args.path == "decode":
+        return run_decode(args, rank, world, local_rank)
 
     import torch
 
