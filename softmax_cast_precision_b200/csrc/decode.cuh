@@ -15,7 +15,10 @@
 //
 // With one query row per head there is no M dimension for the tensor cores:
 // products run on the FP32 pipes.  E4M3 x E4M3 products are exact in FP32.
-// Thread t owns key t of a tile for S = q K^T and output column t for P^ V.
+// Thread t owns key t of a tile for S = q K^T; for P^ V it owns the four
+// output columns 4 (t % 32) .. + 3 over the keys 32 (t / 32) .. + 31 of each
+// tile (one 32-bit load of V per key), and the four key quarters are summed
+// once per split.
 // K rows are stored with their 16-byte chunks XOR-swizzled by (row & 7), so
 // that a warp reading one chunk of 32 different rows hits 32 distinct banks.
 #pragma once
@@ -78,7 +81,7 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
   uint8_t* sK = dsm;                            // 2 x 16 KB, swizzled rows
   uint8_t* sV = dsm + 2 * kTile;                // 2 x 16 KB
   float* sQ = reinterpret_cast<float*>(dsm + 4 * kTile);  // [G][128]
-  float* sP = sQ + kDecodeMaxG * 128;                     // [G][128] P^ values
+  float* sP = sQ + kDecodeMaxG * 128;                     // [128 keys][8] P^ values
   float* sRed = sP + kDecodeMaxG * 128;                   // [4 warps][G]
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int split = blockIdx.x, zkv = blockIdx.y;  // zkv = b * Hkv + hkv
@@ -114,9 +117,13 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
     cp_async_commit();
   };
 
-  float m[kDecodeMaxG], l[kDecodeMaxG], acc[kDecodeMaxG];
+  float m[kDecodeMaxG], l[kDecodeMaxG], acc[kDecodeMaxG][4];
 #pragma unroll
-  for (int g = 0; g < kDecodeMaxG; ++g) m[g] = -INFINITY, l[g] = 0.0f, acc[g] = 0.0f;
+  for (int g = 0; g < kDecodeMaxG; ++g) {
+    m[g] = -INFINITY, l[g] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[g][j] = 0.0f;
+  }
   const float c = p.scale_log2;
 
   fetch(tile_of(0), 0);
@@ -181,7 +188,7 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
         // P * S for key t: the scale enters the exponent; masked keys give 0.
         const float ps = valid ? ex2_approx(fmaf(s[g], c, p.log2_p_scale - m_new)) : 0.0f;
         s[g] = ps;
-        sP[g * 128 + t] = e4m3_round(ps);
+        sP[t * kDecodeMaxG + g] = e4m3_round(ps);
       }
     }
     __syncthreads();  // every thread has read sRed (maxima) and written sP
@@ -194,25 +201,28 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
         if (lane == 0) sRed[warp * kDecodeMaxG + g] = x;
       }
     }
-    // P^ V for output column t.
-    const uint8_t* vcol = sV + buf * kTile + t;
+    // P^ V: columns 4 cg .. 4 cg + 3 over this thread's quarter of the keys.
 #pragma unroll
-    for (int g = 0; g < kDecodeMaxG; ++g) acc[g] *= alpha[g];
+    for (int g = 0; g < kDecodeMaxG; ++g) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[g][j] *= alpha[g];
+    }
+    const uint8_t* vtile = sV + buf * kTile + (lane << 2);
 #pragma unroll 4
-    for (int key = 0; key < 128; key += 4) {
-      const uint32_t w = static_cast<uint32_t>(vcol[key * 128]) | (static_cast<uint32_t>(vcol[(key + 1) * 128]) << 8) |
-                         (static_cast<uint32_t>(vcol[(key + 2) * 128]) << 16) |
-                         (static_cast<uint32_t>(vcol[(key + 3) * 128]) << 24);
+    for (int kk = 0; kk < 32; ++kk) {
+      const int key = (warp << 5) + kk;
       float v0, v1, v2, v3;
-      e4m3x4_to_f32(w, v0, v1, v2, v3);
+      e4m3x4_to_f32(*reinterpret_cast<const uint32_t*>(vtile + key * 128), v0, v1, v2, v3);
+      const float4 pa = *reinterpret_cast<const float4*>(sP + key * kDecodeMaxG);
+      const float4 pb = *reinterpret_cast<const float4*>(sP + key * kDecodeMaxG + 4);
+      const float pg[kDecodeMaxG] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
 #pragma unroll
       for (int g = 0; g < kDecodeMaxG; ++g) {
         if (g < G) {
-          const float* pg = sP + g * 128 + key;
-          acc[g] = fmaf(pg[0], v0, acc[g]);
-          acc[g] = fmaf(pg[1], v1, acc[g]);
-          acc[g] = fmaf(pg[2], v2, acc[g]);
-          acc[g] = fmaf(pg[3], v3, acc[g]);
+          acc[g][0] = fmaf(pg[g], v0, acc[g][0]);
+          acc[g][1] = fmaf(pg[g], v1, acc[g][1]);
+          acc[g][2] = fmaf(pg[g], v2, acc[g][2]);
+          acc[g][3] = fmaf(pg[g], v3, acc[g][3]);
         }
       }
     }
@@ -226,12 +236,24 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
     }
     __syncthreads();  // sRed is rewritten by the next tile's maxima
   }
-  // Partial results of this split.
+  // Sum of the four key quarters (through the K buffers, free now), then
+  // the partial results of this split.
+  float* sAcc = reinterpret_cast<float*>(dsm);  // [4 quarters][G][128]
 #pragma unroll
   for (int g = 0; g < kDecodeMaxG; ++g) {
     if (g < G) {
+      *reinterpret_cast<float4*>(sAcc + (warp * kDecodeMaxG + g) * 128 + (lane << 2)) =
+          make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int g = 0; g < kDecodeMaxG; ++g) {
+    if (g < G) {
+      const float sum = (sAcc[(0 * kDecodeMaxG + g) * 128 + t] + sAcc[(1 * kDecodeMaxG + g) * 128 + t]) +
+                        (sAcc[(2 * kDecodeMaxG + g) * 128 + t] + sAcc[(3 * kDecodeMaxG + g) * 128 + t]);
       float* dst = p.part + (static_cast<int64_t>(b * p.H + hkv * G + g) * p.splits + split) * kDecodePartStride;
-      dst[t] = acc[g];
+      dst[t] = sum;
       if (t == 0) {
         dst[128] = m[g];
         dst[129] = l[g];
