@@ -184,3 +184,26 @@ def test_decode_workspace_and_validation(fp8):
     assert call(S=0.0) == fp8.ERR_INVALID_ARG
     assert call(order=3) == fp8.ERR_INVALID_ARG
     assert call(B=0) == fp8.OK
+
+
+def test_binding_rejects_bad_arguments_before_calling_the_library(fp8):
+    import torch
+
+    b16 = torch.zeros((1, 2, 8, 128), dtype=torch.bfloat16)
+    u8 = torch.zeros((1, 2, 8, 128), dtype=torch.uint8)
+    with pytest.raises(TypeError):
+        fp8.fwd_bf16qk(u8, u8, u8, causal=True)  # q, k must be bfloat16
+    with pytest.raises(ValueError):
+        fp8.fwd_bf16qk(b16, b16, u8, causal=True)  # host tensors
+    with pytest.raises(ValueError):
+        fp8.quantize(b16, 128)  # host tensor
+    with pytest.raises(ValueError):
+        fp8.quantize(torch.zeros((2, 8, 128), dtype=torch.float16), 128)  # host tensor (checked first)
+    with pytest.raises(ValueError):
+        fp8.decode(u8, u8, u8)  # q must be [B, H, d]
+    with pytest.raises(ValueError):
+        fp8.decode(torch.zeros((1, 2, 128), dtype=torch.uint8), u8, u8)  # host tensors
+    with pytest.raises(ValueError):
+        fp8.fwd(u8, u8[:, :1], u8, causal=True, kv_order="sideways")
+    with pytest.raises(ValueError):
+        fp8.fwd_noalloc(u8.cuda() if torch.cuda.is_available() else u8, u8, u8, torch.empty(0), causal=True)
