@@ -81,17 +81,20 @@ def _strip_comments(src: str) -> str:
     return " ".join(code.split())
 
 
+# The device code of the persistent forward kernel (its parameters, PTX
+# wrappers and the kernel itself); the other paths' kernels live elsewhere.
+KERNEL_SOURCES = ("fwd_v1.cuh", "fwd_v2.cuh", "sm100_ptx.cuh")
+
+
 def kernel_source_hash() -> str:
     """Hash of the forward kernel's code and its launch configuration.
 
-    Covers the device headers and the host function that sizes the
-    persistent kernel's launch; insensitive to comments and layout.
+    Covers the device sources of that kernel and the host function that
+    sizes its launch; insensitive to comments and layout.
     """
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "softmax_cast_precision_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if not name.endswith(".cuh"):
-            continue
+    for name in KERNEL_SOURCES:
         with open(os.path.join(csrc, name), encoding="utf-8") as fh:
             h.update(name.encode() + _strip_comments(fh.read()).encode())
     with open(os.path.join(csrc, "api.cu"), encoding="utf-8") as fh:

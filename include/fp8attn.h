@@ -13,15 +13,19 @@
  * "L'algoritmo Flash Attention" and "La ricorrenza softmax online"; causal
  * block skipping is its section on causal masking.
  *
- * Conventions shared by every call:
+ * Conventions shared by the calls (each call's comment states its exceptions):
  *   - All tensor arguments are DEVICE pointers to caller-owned memory; the
  *     library keeps no pointer after a call returns.  Pointers must be
- *     16-byte aligned.  For d = 128 each call takes a 256-byte work-unit
- *     counter from a per-device stream-ordered memory pool the library
- *     creates on first use (cudaMallocFromPoolAsync on the call's stream,
- *     returned with cudaFreeAsync on the same stream before the call
+ *     16-byte aligned (descale and lse arrays: 4-byte).  The rotation signs
+ *     of fp8attn_quantize and fp8attn_fwd_scaled are a HOST array.
+ *   - The persistent-kernel calls (fp8attn_fwd, fp8attn_pzero_count,
+ *     fp8attn_fwd_scaled, fp8attn_fwd_bf16qk at d = 128) each take a 256-byte
+ *     work-unit counter from a per-device stream-ordered memory pool the
+ *     library creates on first use (cudaMallocFromPoolAsync on the call's
+ *     stream, returned with cudaFreeAsync on the same stream before the call
  *     returns; the pool keeps its memory mapped for reuse), so concurrent
- *     calls on different streams are independent.
+ *     calls on different streams are independent.  fp8attn_fwd_noalloc,
+ *     fp8attn_quantize and fp8attn_decode allocate nothing.
  *   - Layouts are contiguous, row-major, with the head dimension innermost:
  *       q    [B, H,   N, d]  E4M3 bytes (OCP E4M3FN)
  *       k, v [B, Hkv, N, d]  E4M3 bytes

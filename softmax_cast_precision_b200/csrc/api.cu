@@ -1,9 +1,10 @@
 // api.cu -- the C ABI of libfp8attn (declared in include/fp8attn.h): argument
-// validation, TMA tensor-map construction and kernel launch.  Every tensor is
-// caller-owned device memory; the only device memory the library touches
-// besides it is a per-call 256-byte scheduler block from the stream-ordered
-// allocator (fp8attn_fwd, d = 128), the module-static scratch array of
-// fp8attn_fwd_noalloc and a module-static error word.
+// validation, TMA tensor-map construction and kernel launch.  Every tensor
+// (the decode workspace included) is caller-owned device memory; the only
+// device memory the library touches besides it is a per-call 256-byte
+// scheduler block from the stream-ordered allocator (the persistent kernel's
+// calls at d = 128), the module-static scratch array of fp8attn_fwd_noalloc
+// and a module-static error word.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
