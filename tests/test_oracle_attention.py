@@ -216,3 +216,25 @@ def test_non_sink_mass_lost_at_sink_strength_7():
         assert FACTS["non_sink_loss_low"] <= loss <= FACTS["non_sink_loss_high"], loss
     r256 = oracle.emulate(q, k, v, causal=False, block_n=128, p_scale=256.0, reverse=True)
     assert abs(1.0 - r256.o_f32[..., 0].sum() / o64[..., 0].sum()) < 0.01
+
+
+def test_scale_sawtooth_in_the_kernel_faithful_setting():
+    # Q, K, V kept in FP32 as in the P-cast summary's experiments (section 3
+    # point 4, section 4).  Reverse order (no collapse), so the error is the
+    # cast's rounding alone.  It follows the normalised step d_p(S) of section
+    # 2 (condition 2): the same on every power of two, higher off the grid
+    # (d_p = 1.33 x 2^-4 at 384, 1.6 x 2^-4 at 320), and at 448 (1.14 x 2^-4)
+    # between the two.
+    N, H, d = int(FACTS["experiment_n"]), 4, 128
+    q, k, v, _ = synthetic.make_wide_inputs(1, H, H, N, d, 7.0, seed=101)
+    o64, _ = oracle.attention_fp64(q, k, v, False)
+
+    def mse(S):
+        r = oracle.emulate(q, k, v, causal=False, block_n=128, p_scale=S, reverse=True)
+        return float(np.mean((r.o_f32.astype(np.float64) - o64) ** 2))
+
+    m = {S: mse(S) for S in (128.0, 256.0, 320.0, 384.0, 448.0)}
+    assert abs(m[128.0] / m[256.0] - 1.0) < 0.01
+    for S in (320.0, 384.0):
+        assert m[S] > 1.08 * m[256.0], (S, m)
+    assert 1.02 * m[256.0] < m[448.0] < m[384.0], m
