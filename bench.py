@@ -67,6 +67,9 @@ def parse_args():
     ap.add_argument("--path", default="fp8", choices=["fp8", "wide", "bf16qk", "decode"],
                     help="fp8: E4M3 inputs (the headline); wide: bfloat16 inputs quantised in the step; "
                          "bf16qk: bfloat16 Q and K, E4M3 V; decode: one query row per head, split-KV")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="replicas: each rank runs its own copy (weak scaling, the default); heads: the ranks "
+                         "split one problem's kv heads and all-gather the output (strong scaling)")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (used under ncu)")
     return ap.parse_args()
@@ -647,6 +650,74 @@ def run_decode(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+def run_sharded(args, rank, world, local_rank):
+    """Strong scaling: one 32K prefill split by kv heads across the ranks; a step
+    is every rank's shard plus the all-gather of O and lse (NCCL)."""
+    import torch
+
+    from softmax_cast_precision_b200 import fp8attn
+    from softmax_cast_precision_b200.parallel import fwd_head_sharded
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    w = WORKLOAD
+    q, k, v, _ = synthetic.workload_inputs(w, seed=SEED)  # the same problem on every rank
+    qd, kd, vd = (torch.from_numpy(x).to(device) for x in (q, k, v))
+    stream = torch.cuda.current_stream(device)
+
+    def shard_fwd(qs, ks, vs, **kw):
+        return fp8attn.fwd(qs, ks, vs, stream=stream, **kw)
+
+    def step():
+        if dist is None:
+            return fp8attn.fwd(qd, kd, vd, causal=w.causal, p_scale=P_SCALE, kv_order=KV_ORDER, stream=stream)
+        return fwd_head_sharded(qd, kd, vd, causal=w.causal, p_scale=P_SCALE, kv_order=KV_ORDER, compute=shard_fwd)
+
+    for _ in range(args.warmup):
+        step()
+    fp8attn.check_error(stream=stream, device=device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local_rank) as clk:
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(device)
+        ev[0].record(stream)
+        for i in range(args.steps):
+            o, lse = step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize(device)
+        if dist is not None:
+            dist.barrier()
+    fp8attn.check_error(stream=stream, device=device)
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), dist, device)
+    ms_per_step = total_ms / args.steps
+    flops = w.flops()
+    mse = mse_vs_fp64(qd, kd, vd, o, sample_rows(w.N, 256)) if rank == 0 else None
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": METRIC, "value": flops / (ms_per_step * 1e-3) / 1e12, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": WORKLOAD_DESC, "flop_per_step": flops, "l2": "inputs exceed L2 (402 MB)",
+                   "parallelism": f"kv heads split over {world} ranks, all-gather of O and lse"},
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+        "mse_vs_fp64": {"value": mse, "rows": "256 evenly spaced query rows of each head",
+                        "reference": "PyTorch float64 softmax(QK^T/sqrt(d))V on the same E4M3 inputs"},
+    }), flush=True)
+
+
 def hbm_peak() -> float:
     try:
         with open(PEAKS_FILE) as fh:
@@ -741,6 +812,10 @@ def main():
         if args.path in ("bf16qk", "decode"):
             raise SystemExit("--impl reference covers --path fp8 and wide")
         return run_reference_wide(args, rank) if args.path == "wide" else run_reference(args, rank, world)
+    if args.shard == "heads":
+        if args.path != "fp8" or args.impl != "ours":
+            raise SystemExit("--shard heads covers the fp8 path")
+        return run_sharded(args, rank, world, local_rank)
     if args.path == "wide":
         return run_wide(args, rank, world, local_rank)
     if args.path == "bf16qk":
