@@ -1,12 +1,17 @@
 """Throughput benchmark of the FP8 (E4M3) P-cast attention forward pass.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--path fp8|wide]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--path fp8|wide|bf16qk|decode] [--shard replicas|heads]
 
 One step is one forward pass of the 32K causal prefill (B=1, H=32, N=32768,
 d=128, Delta=7 sink with k=4, S=256, reverse KV order) through the C ABI.
-Rank 0 prints one JSON line (see the design doc for every key).  Under torchrun
-each rank runs its own copy of the workload on its own GPU (no collective on
-the data path: weak scaling); the step time is the maximum over ranks.
+Rank 0 prints one JSON line: the throughput, the roofline of the dominant
+kernel, the oracle's CPU time, the end-to-end figure with host buffers, the
+SM clocks sampled during the timed region and the count of kernel launches.
+Under torchrun each rank runs its own copy of the workload on its own GPU (no
+collective on the data path: weak scaling); the step time is the maximum over
+ranks.  --shard heads splits one problem's kv heads across the ranks instead
+and all-gathers O and lse (strong scaling).
 
 --impl reference times the CPU oracle (the blockwise E4M3 emulator) on the
 host cores instead, on a bounded sample of the same workload per step.
