@@ -25,7 +25,7 @@
  *     stream, returned with cudaFreeAsync on the same stream before the call
  *     returns; the pool keeps its memory mapped for reuse), so concurrent
  *     calls on different streams are independent.  fp8attn_fwd_noalloc,
- *     fp8attn_quantize and fp8attn_decode allocate nothing.
+ *     fp8attn_quantize, fp8attn_decode and fp8attn_bwd allocate nothing.
  *   - Layouts are contiguous, row-major, with the head dimension innermost:
  *       q    [B, H,   N, d]  E4M3 bytes (OCP E4M3FN)
  *       k, v [B, Hkv, N, d]  E4M3 bytes
@@ -177,6 +177,33 @@ int fp8attn_decode(const void* q, const void* k, const void* v, void* o, float* 
 
 /* Workspace bytes fp8attn_decode needs (0 for invalid sizes). */
 unsigned long long fp8attn_decode_workspace_bytes(int B, int H, int N, int split_tiles);
+
+/*
+ * Backward pass of fp8attn_fwd (experimental: its GPU parity tests against
+ * the oracle are pending).  Given the forward inputs q, k, v (E4M3), its
+ * outputs o (bfloat16 [B, H, N, d]) and lse (float32 [B, H, N], natural log,
+ * as fp8attn_fwd writes it) and the output gradient dout (bfloat16 [B, H, N,
+ * d]), writes the float32 gradients
+ *   dq [B, H, N, d],  dk [B, Hkv, N, d],  dv [B, Hkv, N, d]
+ * and delta [B, H, N], delta_i = dout_i . o_i.  The probabilities are
+ * recomputed from lse, P_ij = exp(q_i.k_j/sqrt(d) - lse_i), as in the
+ * recomputation form of "Attenzione flash e domanda sulla lunghezza della
+ * sequenza"; the P-cast of "P-Cast Precision in FP8 Attention", technical
+ * summary, section 1, is kept where the forward pass applies it:
+ *   dv_j = sum_i E4M3(P_ij S) dout_i / S
+ *   dS_ij = P_ij (dout_i . v_j - delta_i)   (the cast is the identity here)
+ *   dq_i = sum_j dS_ij k_j / sqrt(d),   dk_j = sum_i dS_ij q_i / sqrt(d)
+ * dk and dv sum over the H / Hkv query heads that share a kv head.  dS is
+ * rounded to bfloat16 before its two products; everything else accumulates
+ * in float32.  The gradients do not depend on the forward call's kv_order.
+ * d must be 128 (FP8ATTN_ERR_UNSUPPORTED otherwise); B * H * N at most 2^34.
+ * All pointers are device pointers, caller-owned, 16-byte aligned (lse and
+ * delta: 4-byte); the outputs are overwritten.  Allocates nothing; launches
+ * three kernels on stream (the row dots, then dk and dv, then dq).
+ */
+int fp8attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                const void* dout, float* dq, float* dk, float* dv, float* delta,
+                int B, int H, int Hkv, int N, int d, int causal, float p_scale, void* stream);
 
 /*
  * Allocation-free forward pass.  The pages have no counterpart of this call:

@@ -1,5 +1,6 @@
 // api.cu -- the C ABI of libfp8attn (declared in include/fp8attn.h): argument
-// validation, TMA tensor-map construction and kernel launch.  Every tensor
+// validation, TMA tensor-map construction and kernel launch (forward,
+// quantisation, decode and backward).  Every tensor
 // (the decode workspace included) is caller-owned device memory; the only
 // device memory the library touches besides it is a per-call 256-byte
 // scheduler block from the stream-ordered allocator (the persistent kernel's
@@ -18,6 +19,7 @@
 #include "fwd_v2.cuh"
 #include "quantize.cuh"
 #include "decode.cuh"
+#include "bwd.cuh"
 
 namespace fp8attn {
 
@@ -501,6 +503,60 @@ extern "C" int fp8attn_decode(const void* q, const void* k, const void* v, void*
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   decode_split_kernel<<<dim3(p.splits, B * Hkv), 128, kSmem, s>>>(p);
   decode_combine_kernel<<<B * H, 128, 0, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
+}
+
+extern "C" int fp8attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                           const void* dout, float* dq, float* dk, float* dv, float* delta, int B, int H, int Hkv,
+                           int N, int d, int causal, float p_scale, void* stream) {
+  using namespace fp8attn;
+  if (B < 0 || N < 0 || H < 1 || Hkv < 1 || H % Hkv != 0) return FP8ATTN_ERR_INVALID_ARG;
+  if (d != 128) return FP8ATTN_ERR_UNSUPPORTED;
+  if (!(p_scale >= 0x1p-64f) || !(p_scale <= 0x1p64f)) return FP8ATTN_ERR_INVALID_ARG;
+  if (B > 65535 || H > 65535) return FP8ATTN_ERR_UNSUPPORTED;  // grid y/z limits
+  const int64_t rows = static_cast<int64_t>(B) * H * N;
+  if (rows > (int64_t(1) << 34)) return FP8ATTN_ERR_UNSUPPORTED;  // row-dot grid: rows / 8 blocks
+  if (rows == 0) return FP8ATTN_OK;
+  auto a16 = [](const void* ptr) { return ptr != nullptr && aligned16(ptr); };
+  auto a4 = [](const void* ptr) { return ptr != nullptr && (reinterpret_cast<uintptr_t>(ptr) & 3u) == 0; };
+  if (!a16(q) || !a16(k) || !a16(v) || !a16(o) || !a16(dout) || !a16(dq) || !a16(dk) || !a16(dv) || !a4(lse) ||
+      !a4(delta))
+    return FP8ATTN_ERR_INVALID_ARG;
+  BwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.o = o;
+  p.dout = dout;
+  p.lse = lse;
+  p.delta = delta;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.B = B;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.h_per_kv = H / Hkv;
+  p.causal = causal ? 1 : 0;
+  p.num_tiles = (N + 127) / 128;
+  p.p_scale = p_scale;
+  p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
+  p.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(128.0));
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map(&tq, q, 128, N, B * H, 128) || !make_map(&tk, k, 128, N, B * Hkv, 128) ||
+      !make_map(&tv, v, 128, N, B * Hkv, 128) || !make_map_bf16(&tdo, dout, N, B * H))
+    return FP8ATTN_ERR_CUDA;
+  uint32_t* err_word = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err_word), g_error_word) != cudaSuccess)
+    return FP8ATTN_ERR_CUDA;
+  if (cudaFuncSetAttribute(bwd_dkdv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DkdvLayout::SMEM_BYTES) !=
+          cudaSuccess ||
+      cudaFuncSetAttribute(bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DqLayout::SMEM_BYTES) !=
+          cudaSuccess)
+    return FP8ATTN_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  bwd_delta_kernel<<<static_cast<unsigned int>((rows + 7) / 8), 256, 0, s>>>(p);
+  bwd_dkdv_kernel<<<dim3(p.num_tiles, Hkv, B), 128, DkdvLayout::SMEM_BYTES, s>>>(tq, tk, tv, tdo, p, err_word);
+  bwd_dq_kernel<<<dim3(p.num_tiles, H, B), 128, DqLayout::SMEM_BYTES, s>>>(tq, tk, tv, tdo, p, err_word);
   return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
 }
 

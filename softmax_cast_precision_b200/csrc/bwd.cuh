@@ -1,0 +1,559 @@
+// bwd.cuh -- backward pass of the P-cast attention on sm_100a (d = 128).
+//
+// The gradients are those of the recomputation form of "Attenzione flash e
+// domanda sulla lunghezza della sequenza" (FlashAttention keeps O and the
+// log-sum-exp and recomputes P from them), with the P-cast of "P-Cast
+// Precision in FP8 Attention", technical summary, section 1, kept where the
+// forward pass applies it, on the probabilities that multiply V:
+//
+//   P_ij  = exp(s_ij - lse_i),  s_ij = q_i . k_j / sqrt(d)   (masked: 0)
+//   dV_j  = sum_i E4M3(P_ij S) dO_i / S
+//   dP_ij = dO_i . v_j,   D_i = dO_i . O_i,   dS_ij = P_ij (dP_ij - D_i)
+//   dQ_i  = sum_j dS_ij k_j / sqrt(d),   dK_j = sum_i dS_ij q_i / sqrt(d)
+//
+// The cast is the identity for differentiation (dS uses the unquantised P).
+//
+// Three kernels, all on the caller's stream:
+//   bwd_delta_kernel  D_i = dO_i . O_i (one warp per row);
+//   bwd_dkdv_kernel   one CTA per (batch, kv head, 128-key tile): for every
+//                     query head of the group and every query tile that sees
+//                     the keys, S^T = K Q^T and dP^T = V dO^T on the tensor
+//                     cores, P^T, E4M3(P^T S) and dS^T in registers, then
+//                     dV += E4M3(P^T S) dO and dK += dS^T Q accumulated in
+//                     tensor memory; no atomics (the group's heads are summed
+//                     in the CTA);
+//   bwd_dq_kernel     one CTA per (batch, head, 128-row query tile): S and dP
+//                     recomputed per key tile, dQ += dS K in tensor memory.
+//
+// Operands.  Q, K and V are E4M3 and dO is bfloat16.  S (S^T) multiplies two
+// E4M3 tiles (kind::f8f6f4).  The products with dO or dS take both operands
+// in bfloat16 (kind::f16): the E4M3 tiles are converted in shared memory,
+// exactly (every E4M3 value is a bfloat16 value), and so are the cast
+// probabilities E4M3(P S); dS is rounded to bfloat16 (nearest even).  Every
+// 16-bit tile is 128 rows x 128 columns stored as two 64-column panels under
+// the 128-byte swizzle (16 KB apart), the layout a TMA box of 64 bfloat16
+// columns writes; the MMAs read it K-major (K along the row) or MN-major (M
+// or N along the row) as each product needs.  Accumulators are FP32 in
+// tensor memory and the gradients are written in FP32.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace fp8attn {
+
+struct BwdParams {
+  const void* o;       // bf16 [B, H, N, 128]
+  const void* dout;    // bf16 [B, H, N, 128]
+  const float* lse;    // f32  [B, H, N], natural log
+  float* delta;        // f32  [B, H, N]: D_i (written by bwd_delta_kernel)
+  float* dq;           // f32  [B, H, N, 128]
+  float* dk;           // f32  [B, Hkv, N, 128]
+  float* dv;           // f32  [B, Hkv, N, 128]
+  int B, H, Hkv, N;
+  int h_per_kv;        // H / Hkv
+  int causal;
+  int num_tiles;       // ceil(N / 128), query and key tiles alike
+  float p_scale;       // S
+  float scale_log2;    // log2(e) / sqrt(128)
+  float inv_sqrt_d;    // 1 / sqrt(128)
+};
+
+struct BwdConfig {
+  static constexpr int T = 128;                   // rows of every tile (queries or keys)
+  static constexpr int F8_TILE = T * 128;         // one E4M3 tile: 16 KB
+  static constexpr int BF_PANEL = T * 128;        // one 64-column bfloat16 panel: 16 KB
+  static constexpr int BF_TILE = 2 * BF_PANEL;    // one bfloat16 tile: 32 KB
+  static constexpr uint32_t TMEM_COLS = 512;
+};
+
+// Shared-memory layout of bwd_dkdv_kernel (offsets from a 1024-byte aligned base).
+struct DkdvLayout {
+  static constexpr int OFF_K = 0;                                   // K_j   E4M3
+  static constexpr int OFF_VF = OFF_K + BwdConfig::F8_TILE;         // V_j   E4M3 (converted once)
+  static constexpr int OFF_VB = OFF_VF + BwdConfig::F8_TILE;        // V_j   bf16
+  static constexpr int OFF_Q = OFF_VB + BwdConfig::BF_TILE;         // Q_i   E4M3
+  static constexpr int OFF_QB = OFF_Q + BwdConfig::F8_TILE;         // Q_i   bf16
+  static constexpr int OFF_DO = OFF_QB + BwdConfig::BF_TILE;        // dO_i  bf16
+  static constexpr int OFF_PT = OFF_DO + BwdConfig::BF_TILE;        // E4M3(P^T S) as bf16
+  static constexpr int OFF_DST = OFF_PT + BwdConfig::BF_TILE;       // dS^T  bf16
+  static constexpr int OFF_VEC = OFF_DST + BwdConfig::BF_TILE;      // lse_i * log2(e) [128], D_i [128]
+  static constexpr int OFF_BAR = OFF_VEC + 2 * 128 * 4;
+  static constexpr int SMEM_BYTES = OFF_BAR + 128 + 1024;           // barriers, TMEM slot, alignment slack
+};
+
+// Shared-memory layout of bwd_dq_kernel.
+struct DqLayout {
+  static constexpr int OFF_Q = 0;                                   // Q_i   E4M3
+  static constexpr int OFF_DO = OFF_Q + BwdConfig::F8_TILE;         // dO_i  bf16
+  static constexpr int OFF_K = OFF_DO + BwdConfig::BF_TILE;         // K_j   E4M3
+  static constexpr int OFF_V = OFF_K + BwdConfig::F8_TILE;          // V_j   E4M3
+  static constexpr int OFF_KB = OFF_V + BwdConfig::F8_TILE;         // K_j   bf16
+  static constexpr int OFF_VB = OFF_KB + BwdConfig::BF_TILE;        // V_j   bf16
+  static constexpr int OFF_DS = OFF_VB + BwdConfig::BF_TILE;        // dS    bf16
+  static constexpr int OFF_BAR = OFF_DS + BwdConfig::BF_TILE;
+  static constexpr int SMEM_BYTES = OFF_BAR + 128 + 1024;
+};
+
+// Instruction descriptor for kind::f16 with bfloat16 A and B and an FP32
+// accumulator, with the operand majors given (bit 15: A MN-major, bit 16: B
+// MN-major).
+__host__ __device__ constexpr uint32_t bwd_idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn_major) << 15) |
+         (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Byte offset of 16-byte chunk `c` (0..15, eight bfloat16 columns each) of
+// row `r` in a two-panel bfloat16 tile: panel c / 8, chunk c % 8 of the
+// panel's 128-byte row, XORed with r % 8 (the 128-byte swizzle).
+__device__ __forceinline__ uint32_t bf16_tile_chunk(int r, int c) {
+  return static_cast<uint32_t>((c >> 3) * BwdConfig::BF_PANEL + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+// Four E4M3 codes (one 32-bit word, lowest byte first) to four bfloat16
+// values in two words (exact: E4M3 -> f16 -> f32 -> bf16 loses nothing).
+__device__ __forceinline__ uint2 bwd_e4m3x4_to_bf16x4(uint32_t w) {
+  uint32_t lo, hi;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(lo) : "h"(static_cast<uint16_t>(w & 0xFFFFu)));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hi) : "h"(static_cast<uint16_t>(w >> 16)));
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&hi));
+  return make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(b.x, b.y));
+}
+
+// Row `r` of an E4M3 tile (128 bytes per row, 128-byte swizzle, as TMA wrote
+// it) into row `r` of a two-panel bfloat16 tile.
+__device__ __forceinline__ void bwd_convert_row(const uint8_t* src, uint8_t* dst, int r) {
+  const uint32_t s = smem_u32(src), d = smem_u32(dst);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint32_t w0, w1, w2, w3;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+                 : "r"(s + r * 128 + ((c ^ (r & 7)) << 4))
+                 : "memory");
+    // 16 E4M3 columns 16c .. 16c+15 become bfloat16 chunks 2c and 2c+1.
+    const uint2 a = bwd_e4m3x4_to_bf16x4(w0), b = bwd_e4m3x4_to_bf16x4(w1);
+    const uint2 e = bwd_e4m3x4_to_bf16x4(w2), f = bwd_e4m3x4_to_bf16x4(w3);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d + bf16_tile_chunk(r, 2 * c)), "r"(a.x),
+                 "r"(a.y), "r"(b.x), "r"(b.y)
+                 : "memory");
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d + bf16_tile_chunk(r, 2 * c + 1)), "r"(e.x),
+                 "r"(e.y), "r"(f.x), "r"(f.y)
+                 : "memory");
+  }
+}
+
+// Stores 32 FP32 values (columns 32*g .. 32*g+31 of row `r`) as bfloat16
+// chunks 4g .. 4g+3 of a two-panel tile.
+__device__ __forceinline__ void bwd_store_bf16_32(uint8_t* dst, int r, int g, const float (&x)[32]) {
+  const uint32_t d = smem_u32(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const uint32_t w0 = pack_bf16x2(x[8 * q + 0], x[8 * q + 1]);
+    const uint32_t w1 = pack_bf16x2(x[8 * q + 2], x[8 * q + 3]);
+    const uint32_t w2 = pack_bf16x2(x[8 * q + 4], x[8 * q + 5]);
+    const uint32_t w3 = pack_bf16x2(x[8 * q + 6], x[8 * q + 7]);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d + bf16_tile_chunk(r, 4 * g + q)), "r"(w0),
+                 "r"(w1), "r"(w2), "r"(w3)
+                 : "memory");
+  }
+}
+
+// The E4M3 value nearest to x (nearest even, saturating), as float32.
+__device__ __forceinline__ float bwd_e4m3_value(float x) {
+  const uint32_t code = cvt_e4m3x2(x, 0.0f);
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(code)));
+  return __low2float(*reinterpret_cast<const __half2*>(&h));
+}
+
+// Descriptors of the three operand forms (start address, LBO, SBO, 128-byte
+// swizzle), with the per-step start-address advance of a K step:
+//   E4M3 tile, K-major:     32 columns = 32 bytes per step (+2 in the >> 4 field);
+//   (kmajor_desc serves both K-major forms: only the step differs)
+//   bf16 tile, K-major:     16 columns = 32 bytes (+2), four steps per panel,
+//                           then the next panel (+16 KB);
+//   bf16 tile, MN-major:    16 rows = 2048 bytes (+128); the N (or M) extent of
+//                           128 spans both panels, LBO = 16 KB apart.
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t saddr) { return smem_desc(saddr, 16, 1024, 2); }
+__device__ __forceinline__ uint64_t bf16_kmajor_step(int kk) {
+  return static_cast<uint64_t>((kk >> 2) * (BwdConfig::BF_PANEL >> 4) + 2 * (kk & 3));
+}
+__device__ __forceinline__ uint64_t bf16_mnmajor_desc(uint32_t saddr) {
+  return smem_desc(saddr, BwdConfig::BF_PANEL, 1024, 2);
+}
+
+// --------------------------------------------------------------------------
+// D_i = dO_i . O_i in FP32, one warp per row (4 columns per lane).
+// --------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) bwd_delta_kernel(const BwdParams p) {
+  const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.N;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint2 a = reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.dout) + row * 128)[lane];
+  const uint2 b = reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(p.o) + row * 128)[lane];
+  auto lo = [](uint32_t w) { return __uint_as_float(w << 16); };
+  auto hi = [](uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); };
+  float s = lo(a.x) * lo(b.x);
+  s = fmaf(hi(a.x), hi(b.x), s);
+  s = fmaf(lo(a.y), lo(b.y), s);
+  s = fmaf(hi(a.y), hi(b.y), s);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (lane == 0) p.delta[row] = s;
+}
+
+// --------------------------------------------------------------------------
+// dK and dV: one CTA (one warpgroup) per (batch, kv head, key tile).
+// --------------------------------------------------------------------------
+__global__ void __launch_bounds__(128, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p, uint32_t* err_word) {
+  using L = DkdvLayout;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* sLse2 = reinterpret_cast<float*>(base + L::OFF_VEC);
+  float* sDelta = sLse2 + 128;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
+  uint64_t* bar_kv = bars + 0;  // K_j and V_j landed
+  uint64_t* bar_q = bars + 1;   // Q_i and dO_i landed
+  uint64_t* bar_s = bars + 2;   // S^T and dP^T computed
+  uint64_t* bar_g = bars + 3;   // dV and dK products of this step complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int jt = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int k0 = jt * 128;
+  const int zkv = b * p.Hkv + hk;
+  const int i_first = p.causal ? jt : 0;  // query tiles before the key tile see none of its keys
+  const int per_head = p.num_tiles - i_first;
+  const int n_iter = p.h_per_kv * per_head;
+
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, BwdConfig::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+
+  auto step_geom = [&](int it, int& zq, int& q0) {
+    const int hl = it / per_head;
+    q0 = (i_first + (it - hl * per_head)) * 128;
+    zq = b * p.H + hk * p.h_per_kv + hl;
+  };
+  auto issue_q = [&](int it) {
+    int zq, q0;
+    step_geom(it, zq, q0);
+    mbar_arrive_expect_tx(bar_q, BwdConfig::F8_TILE + BwdConfig::BF_TILE);
+    tma_load_3d(base + L::OFF_Q, &tm_q, bar_q, 0, q0, zq);
+    tma_load_3d(base + L::OFF_DO, &tm_do, bar_q, 0, q0, zq);
+    tma_load_3d(base + L::OFF_DO + BwdConfig::BF_PANEL, &tm_do, bar_q, 64, q0, zq);
+  };
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar_kv, 2 * BwdConfig::F8_TILE);
+    tma_load_3d(base + L::OFF_K, &tm_k, bar_kv, 0, k0, zkv);
+    tma_load_3d(base + L::OFF_VF, &tm_v, bar_kv, 0, k0, zkv);
+    issue_q(0);
+  }
+
+  const uint32_t sK = smem_u32(base + L::OFF_K), sVB = smem_u32(base + L::OFF_VB);
+  const uint32_t sQ = smem_u32(base + L::OFF_Q), sQB = smem_u32(base + L::OFF_QB);
+  const uint32_t sDO = smem_u32(base + L::OFF_DO), sPT = smem_u32(base + L::OFF_PT);
+  const uint32_t sDST = smem_u32(base + L::OFF_DST);
+  constexpr uint32_t idesc_s = idesc_e4m3_f32(128, 128, false, false);      // S^T = K Q^T
+  constexpr uint32_t idesc_dp = bwd_idesc_bf16(128, 128, false, false);     // dP^T = V dO^T
+  constexpr uint32_t idesc_grad = bwd_idesc_bf16(128, 128, false, true);    // dV += P^T dO, dK += dS^T Q
+
+  const int key = k0 + tid;  // this thread's TMEM lane: one key
+  bool fail = !mbar_wait_bounded(bar_kv, 0, err_word, kErrTimeoutKV);
+  if (!fail) bwd_convert_row(base + L::OFF_VF, base + L::OFF_VB, tid);
+  bool abort = false;
+
+  for (int it = 0; it < n_iter; ++it) {
+    int zq, q0;
+    step_geom(it, zq, q0);
+    {
+      const int qi = q0 + tid;
+      const int64_t idx = static_cast<int64_t>(zq) * p.N + qi;
+      sLse2[tid] = qi < p.N ? p.lse[idx] * 1.4426950408889634f : 0.0f;
+      sDelta[tid] = qi < p.N ? p.delta[idx] : 0.0f;
+    }
+    if (!fail && !mbar_wait_bounded(bar_q, it & 1, err_word, kErrTimeoutQ)) fail = true;
+    if (!fail) bwd_convert_row(base + L::OFF_Q, base + L::OFF_QB, tid);
+    fence_proxy_async_smem();
+    tc_fence_before();
+    abort = __syncthreads_or(fail) != 0;
+    if (abort) break;
+
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_f8_ss(tS, kmajor_desc(sK) + 2 * kk, kmajor_desc(sQ) + 2 * kk, idesc_s, kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ss(tDP, kmajor_desc(sVB) + bf16_kmajor_step(kk), kmajor_desc(sDO) + bf16_kmajor_step(kk),
+                    idesc_dp, kk > 0);
+      mma_commit(bar_s);
+    }
+    if (!mbar_wait_bounded(bar_s, it & 1, err_word, kErrTimeoutMMA)) fail = true;
+    tc_fence_after();
+
+    // P^T, E4M3(P^T S) and dS^T for this thread's key, 32 queries at a time.
+#pragma unroll 1
+    for (int g = 0; g < 4; ++g) {
+      uint32_t rs[32], rdp[32];
+      tmem_ld32(tS + lane_off + 32 * g, rs);
+      tmem_ld32(tDP + lane_off + 32 * g, rdp);
+      tmem_wait_ld();
+      float ph[32], ds[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int c = 32 * g + e;
+        const int qi = q0 + c;
+        const bool visible = qi < p.N && key < p.N && (!p.causal || key <= qi);
+        const float pr = visible ? ex2_approx(__uint_as_float(rs[e]) * p.scale_log2 - sLse2[c]) : 0.0f;
+        ph[e] = bwd_e4m3_value(pr * p.p_scale);
+        ds[e] = pr * (__uint_as_float(rdp[e]) - sDelta[c]);
+      }
+      bwd_store_bf16_32(base + L::OFF_PT, tid, g, ph);
+      bwd_store_bf16_32(base + L::OFF_DST, tid, g, ds);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    abort = __syncthreads_or(fail) != 0;
+    if (abort) break;
+
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const bool acc = (it > 0) || (kk > 0);
+        mma_bf16_ss(tDV, kmajor_desc(sPT) + bf16_kmajor_step(kk), bf16_mnmajor_desc(sDO) + 128 * kk, idesc_grad,
+                    acc);
+        mma_bf16_ss(tDK, kmajor_desc(sDST) + bf16_kmajor_step(kk), bf16_mnmajor_desc(sQB) + 128 * kk,
+                    idesc_grad, acc);
+      }
+      mma_commit(bar_g);
+    }
+    if (!mbar_wait_bounded(bar_g, it & 1, err_word, kErrTimeoutMMA)) fail = true;
+    tc_fence_after();
+    // Q, dO and the converted tiles are free again: fetch the next step's.
+    if (tid == 0 && !fail && it + 1 < n_iter) issue_q(it + 1);
+  }
+  abort = __syncthreads_or(fail || abort) != 0;
+
+  if (!abort) {
+    // Every lane takes part in the warp-wide TMEM loads; lanes past N store nothing.
+    const int64_t row = static_cast<int64_t>(zkv) * p.N + key;
+    float* dvrow = p.dv + row * 128;
+    float* dkrow = p.dk + row * 128;
+#pragma unroll 1
+    for (int g = 0; g < 4; ++g) {
+      uint32_t a[32], c[32];
+      tmem_ld32(tDV + lane_off + 32 * g, a);
+      tmem_ld32(tDK + lane_off + 32 * g, c);
+      tmem_wait_ld();
+      if (key < p.N) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          reinterpret_cast<float4*>(dvrow + 32 * g)[e / 4] = make_float4(
+              __fdiv_rn(__uint_as_float(a[e]), p.p_scale), __fdiv_rn(__uint_as_float(a[e + 1]), p.p_scale),
+              __fdiv_rn(__uint_as_float(a[e + 2]), p.p_scale), __fdiv_rn(__uint_as_float(a[e + 3]), p.p_scale));
+          reinterpret_cast<float4*>(dkrow + 32 * g)[e / 4] =
+              make_float4(__uint_as_float(c[e]) * p.inv_sqrt_d, __uint_as_float(c[e + 1]) * p.inv_sqrt_d,
+                          __uint_as_float(c[e + 2]) * p.inv_sqrt_d, __uint_as_float(c[e + 3]) * p.inv_sqrt_d);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BwdConfig::TMEM_COLS);
+  }
+}
+
+// --------------------------------------------------------------------------
+// dQ: one CTA (one warpgroup) per (batch, head, query tile).
+// --------------------------------------------------------------------------
+__global__ void __launch_bounds__(128, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const BwdParams p, uint32_t* err_word) {
+  using L = DqLayout;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
+  uint64_t* bar_q = bars + 0;   // Q_i and dO_i landed
+  uint64_t* bar_kv = bars + 1;  // K_j and V_j landed
+  uint64_t* bar_s = bars + 2;   // S and dP computed
+  uint64_t* bar_g = bars + 3;   // dQ product of this step complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int it_q = p.num_tiles - 1 - static_cast<int>(blockIdx.x);  // longest causal rows first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int q0 = it_q * 128;
+  const int zq = b * p.H + h;
+  const int zkv = b * p.Hkv + h / p.h_per_kv;
+  const int last = p.causal ? it_q : p.num_tiles - 1;  // key tiles 0 .. last
+
+  if (tid == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, BwdConfig::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 256;
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+
+  auto issue_kv = [&](int j) {
+    mbar_arrive_expect_tx(bar_kv, 2 * BwdConfig::F8_TILE);
+    tma_load_3d(base + L::OFF_K, &tm_k, bar_kv, 0, j * 128, zkv);
+    tma_load_3d(base + L::OFF_V, &tm_v, bar_kv, 0, j * 128, zkv);
+  };
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar_q, BwdConfig::F8_TILE + BwdConfig::BF_TILE);
+    tma_load_3d(base + L::OFF_Q, &tm_q, bar_q, 0, q0, zq);
+    tma_load_3d(base + L::OFF_DO, &tm_do, bar_q, 0, q0, zq);
+    tma_load_3d(base + L::OFF_DO + BwdConfig::BF_PANEL, &tm_do, bar_q, 64, q0, zq);
+    issue_kv(0);
+  }
+
+  const uint32_t sQ = smem_u32(base + L::OFF_Q), sDO = smem_u32(base + L::OFF_DO);
+  const uint32_t sK = smem_u32(base + L::OFF_K), sKB = smem_u32(base + L::OFF_KB);
+  const uint32_t sVB = smem_u32(base + L::OFF_VB), sDS = smem_u32(base + L::OFF_DS);
+  constexpr uint32_t idesc_s = idesc_e4m3_f32(128, 128, false, false);   // S = Q K^T
+  constexpr uint32_t idesc_dp = bwd_idesc_bf16(128, 128, false, false);  // dP = dO V^T
+  constexpr uint32_t idesc_dq = bwd_idesc_bf16(128, 128, false, true);   // dQ += dS K
+
+  const int row = q0 + tid;  // this thread's TMEM lane: one query
+  const int64_t ridx = static_cast<int64_t>(zq) * p.N + row;
+  const float lse2 = row < p.N ? p.lse[ridx] * 1.4426950408889634f : 0.0f;
+  const float dlt = row < p.N ? p.delta[ridx] : 0.0f;
+  bool fail = !mbar_wait_bounded(bar_q, 0, err_word, kErrTimeoutQ);
+  bool abort = false;
+
+  for (int j = 0; j <= last; ++j) {
+    const int j0 = j * 128;
+    if (!fail && !mbar_wait_bounded(bar_kv, j & 1, err_word, kErrTimeoutKV)) fail = true;
+    if (!fail) {
+      bwd_convert_row(base + L::OFF_K, base + L::OFF_KB, tid);
+      bwd_convert_row(base + L::OFF_V, base + L::OFF_VB, tid);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    abort = __syncthreads_or(fail) != 0;
+    if (abort) break;
+
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_f8_ss(tS, kmajor_desc(sQ) + 2 * kk, kmajor_desc(sK) + 2 * kk, idesc_s, kk > 0);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ss(tDP, kmajor_desc(sDO) + bf16_kmajor_step(kk), kmajor_desc(sVB) + bf16_kmajor_step(kk),
+                    idesc_dp, kk > 0);
+      mma_commit(bar_s);
+    }
+    if (!mbar_wait_bounded(bar_s, j & 1, err_word, kErrTimeoutMMA)) fail = true;
+    tc_fence_after();
+    // The E4M3 K and V tiles have been read (S, and the conversions before
+    // the barrier): fetch the next key tile while this one is finished.
+    if (tid == 0 && !fail && j < last) issue_kv(j + 1);
+
+#pragma unroll 1
+    for (int g = 0; g < 4; ++g) {
+      uint32_t rs[32], rdp[32];
+      tmem_ld32(tS + lane_off + 32 * g, rs);
+      tmem_ld32(tDP + lane_off + 32 * g, rdp);
+      tmem_wait_ld();
+      float ds[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        const int kj = j0 + 32 * g + e;
+        const bool visible = row < p.N && kj < p.N && (!p.causal || kj <= row);
+        const float pr = visible ? ex2_approx(__uint_as_float(rs[e]) * p.scale_log2 - lse2) : 0.0f;
+        ds[e] = pr * (__uint_as_float(rdp[e]) - dlt);
+      }
+      bwd_store_bf16_32(base + L::OFF_DS, tid, g, ds);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    abort = __syncthreads_or(fail) != 0;
+    if (abort) break;
+
+    if (tid == 0) {
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        mma_bf16_ss(tDQ, kmajor_desc(sDS) + bf16_kmajor_step(kk), bf16_mnmajor_desc(sKB) + 128 * kk, idesc_dq,
+                    (j > 0) || (kk > 0));
+      mma_commit(bar_g);
+    }
+    // The next step rewrites the converted tiles and dS: wait for this product.
+    if (!mbar_wait_bounded(bar_g, j & 1, err_word, kErrTimeoutMMA)) fail = true;
+    tc_fence_after();
+  }
+  abort = __syncthreads_or(fail || abort) != 0;
+
+  if (!abort) {
+    float* dqrow = p.dq + ridx * 128;
+#pragma unroll 1
+    for (int g = 0; g < 4; ++g) {
+      uint32_t a[32];
+      tmem_ld32(tDQ + lane_off + 32 * g, a);
+      tmem_wait_ld();
+      if (row < p.N) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          reinterpret_cast<float4*>(dqrow + 32 * g)[e / 4] =
+              make_float4(__uint_as_float(a[e]) * p.inv_sqrt_d, __uint_as_float(a[e + 1]) * p.inv_sqrt_d,
+                          __uint_as_float(a[e + 2]) * p.inv_sqrt_d, __uint_as_float(a[e + 3]) * p.inv_sqrt_d);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BwdConfig::TMEM_COLS);
+  }
+}
+
+}  // namespace fp8attn

@@ -1,6 +1,6 @@
 """Python binding of libfp8attn (argument marshalling only).
 
-Every step of the attention forward pass runs in the CUDA library; this module
+Every step of the attention passes runs in the CUDA library; this module
 turns torch tensors into pointers, sizes and a stream, calls the C ABI, and
 turns status codes into exceptions.  PyTorch supplies device memory, streams
 and (for host inputs) the host<->device copies.
@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.fp8attn_decode.restype = i32
         L.fp8attn_decode_workspace_bytes.argtypes = [i32, i32, i32, i32]
         L.fp8attn_decode_workspace_bytes.restype = u64
+        L.fp8attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, P]
+        L.fp8attn_bwd.restype = i32
         L.fp8attn_pzero_count.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, P]
         L.fp8attn_pzero_count.restype = i32
         L.fp8attn_kv_tile.argtypes = [i32]
@@ -233,6 +235,37 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, p_scale: float 
     if st != OK:
         raise Fp8AttnError(st, "fp8attn_decode")
     return o, lse
+
+
+def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
+        dout: torch.Tensor, *, causal: bool, p_scale: float = 256.0, stream=None):
+    """Backward pass of ``fwd`` (experimental; see fp8attn_bwd): gradients of the P-cast attention.
+
+    q, k, v are the forward's E4M3 inputs, o (bfloat16 [B,H,N,d]) and lse
+    (float32 [B,H,N]) its outputs, dout the bfloat16 output gradient; all on
+    one GPU.  Returns (dq [B,H,N,d], dk [B,Hkv,N,d], dv [B,Hkv,N,d], delta
+    [B,H,N]), all float32, delta_i = dout_i . o_i.
+    """
+    q, k, v = _bytes(q), _bytes(k), _bytes(v)
+    B, H, Hkv, N, d = _shapes(q, k, v)
+    if not q.is_cuda or any(t.device != q.device for t in (k, v, o, lse, dout)):
+        raise ValueError("bwd takes device tensors on one device")
+    if o.dtype != torch.bfloat16 or dout.dtype != torch.bfloat16 or lse.dtype != torch.float32:
+        raise TypeError("o and dout must be bfloat16, lse float32")
+    if tuple(o.shape) != (B, H, N, d) or tuple(dout.shape) != (B, H, N, d) or tuple(lse.shape) != (B, H, N):
+        raise ValueError("o and dout must be [B,H,N,d] and lse [B,H,N]")
+    o, lse, dout = o.contiguous(), lse.contiguous(), dout.contiguous()
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty((B, H, N, d), **f32)
+    dk = torch.empty((B, Hkv, N, d), **f32)
+    dv = torch.empty((B, Hkv, N, d), **f32)
+    delta = torch.empty((B, H, N), **f32)
+    st = lib().fp8attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                           _ptr(delta), B, H, Hkv, N, d, int(bool(causal)), ctypes.c_float(p_scale),
+                           _stream_ptr(q.device, stream))
+    if st != OK:
+        raise Fp8AttnError(st, "fp8attn_bwd")
+    return dq, dk, dv, delta
 
 
 def _host_signs(signs, d: int):

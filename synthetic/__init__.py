@@ -162,6 +162,12 @@ def make_wide_inputs(B: int, H: int, Hkv: int, N: int, d: int, delta, seed: int,
     return _to_bf16_values(q), _to_bf16_values(k), _to_bf16_values(v), deltas
 
 
+def make_output_grad(shape, seed: int) -> np.ndarray:
+    """A seeded output gradient dO: standard-normal float32 values rounded to bfloat16."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return _to_bf16_values(rng.standard_normal(shape, dtype=np.float32))
+
+
 def hadamard_signs(d: int, seed: int) -> np.ndarray:
     """The random +-1 column signs of the rotation (float32 [d]), from a seeded generator."""
     rng = np.random.Generator(np.random.PCG64(seed))

@@ -32,7 +32,7 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ["fp8attn_fwd", "fp8attn_fwd_noalloc", "fp8attn_fwd_scaled", "fp8attn_quantize",
                      "fp8attn_fwd_bf16qk", "fp8attn_decode", "fp8attn_decode_workspace_bytes",
-                     "fp8attn_pzero_count", "fp8attn_kv_tile", "fp8attn_status_str",
+                     "fp8attn_bwd", "fp8attn_pzero_count", "fp8attn_kv_tile", "fp8attn_status_str",
                      "fp8attn_check_error"]:
         assert required in names
 
@@ -207,3 +207,41 @@ def test_binding_rejects_bad_arguments_before_calling_the_library(fp8):
         fp8.fwd(u8, u8[:, :1], u8, causal=True, kv_order="sideways")
     with pytest.raises(ValueError):
         fp8.fwd_noalloc(u8.cuda() if torch.cuda.is_available() else u8, u8, u8, torch.empty(0), causal=True)
+
+
+def test_bwd_validation(fp8):
+    """fp8attn_bwd rejects bad sizes, scales, pointers and alignments before any CUDA call."""
+    L = fp8.lib()
+    P = ctypes.c_void_p
+
+    def call(d=128, B=1, H=8, Hkv=2, N=300, S=256.0, q=16, o=16, lse=16, dq=16, delta=16):
+        return L.fp8attn_bwd(P(q), P(16), P(16), P(o), P(lse), P(16), P(dq), P(16), P(16), P(delta), B, H, Hkv, N,
+                             d, 1, ctypes.c_float(S), P(0))
+    assert call(d=64) == fp8.ERR_UNSUPPORTED
+    assert call(H=6, Hkv=4) == fp8.ERR_INVALID_ARG
+    assert call(Hkv=0) == fp8.ERR_INVALID_ARG
+    assert call(N=-1) == fp8.ERR_INVALID_ARG
+    assert call(S=0.0) == fp8.ERR_INVALID_ARG
+    assert call(S=float("nan")) == fp8.ERR_INVALID_ARG
+    assert call(S=2.0 ** 65) == fp8.ERR_INVALID_ARG
+    assert call(B=70000) == fp8.ERR_UNSUPPORTED
+    assert call(B=65535, H=65535, Hkv=65535, N=8) == fp8.ERR_UNSUPPORTED  # more than 2^34 rows
+    assert call(q=0) == fp8.ERR_INVALID_ARG
+    assert call(q=8) == fp8.ERR_INVALID_ARG  # not 16-byte aligned
+    assert call(o=24) == fp8.ERR_INVALID_ARG
+    assert call(dq=0) == fp8.ERR_INVALID_ARG
+    assert call(lse=2) == fp8.ERR_INVALID_ARG
+    assert call(delta=0) == fp8.ERR_INVALID_ARG
+    assert call(B=0) == fp8.OK and call(N=0) == fp8.OK  # empty problems launch nothing
+
+
+def test_bwd_binding_checks(fp8):
+    import torch
+
+    u8 = torch.zeros((1, 2, 8, 128), dtype=torch.uint8)
+    b16 = torch.zeros((1, 2, 8, 128), dtype=torch.bfloat16)
+    lse = torch.zeros((1, 2, 8), dtype=torch.float32)
+    with pytest.raises(ValueError):
+        fp8.bwd(u8, u8, u8, b16, lse, b16, causal=True)  # host tensors
+    with pytest.raises(ValueError):
+        fp8.bwd(u8, u8[:, :, :4], u8, b16, lse, b16, causal=True)  # k disagrees on N
