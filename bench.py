@@ -1,7 +1,7 @@
 """Throughput benchmark of the FP8 (E4M3) P-cast attention forward pass.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--path fp8|wide|bf16qk|decode] [--shard replicas|heads]
+                    [--path fp8|wide|bf16qk|decode|bwd] [--shard replicas|heads]
 
 One step is one forward pass of the 32K causal prefill (B=1, H=32, N=32768,
 d=128, Delta=7 sink with k=4, S=256, reverse KV order) through the C ABI.
@@ -25,6 +25,9 @@ path) with E4M3 V: the P-cast summary's kernel-faithful setting.
 
 --path decode times the split-KV decode pass (B=32, H=32, Hkv=8, N=32768,
 one query row per head, 16-tile splits) against the HBM roofline.
+
+--path bwd times the backward pass of the 32K prefill (dQ, dK, dV from the
+forward's inputs, O, lse and a bfloat16 dO).
 """
 from __future__ import annotations
 
@@ -69,9 +72,10 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--path", default="fp8", choices=["fp8", "wide", "bf16qk", "decode"],
+    ap.add_argument("--path", default="fp8", choices=["fp8", "wide", "bf16qk", "decode", "bwd"],
                     help="fp8: E4M3 inputs (the headline); wide: bfloat16 inputs quantised in the step; "
-                         "bf16qk: bfloat16 Q and K, E4M3 V; decode: one query row per head, split-KV")
+                         "bf16qk: bfloat16 Q and K, E4M3 V; decode: one query row per head, split-KV; "
+                         "bwd: the backward pass of the 32K prefill")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="replicas: each rank runs its own copy (weak scaling, the default); heads: the ranks "
                          "split one problem's kv heads and all-gather the output (strong scaling)")
@@ -655,6 +659,136 @@ def run_decode(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+BWD_WORKLOAD_DESC = ("prefill32k backward: B=1 H=32 N=32768 d=128 causal, E4M3 Q/K/V (Delta=7 sink, k=4), "
+                     "O and lse from fp8attn_fwd (S=256, reverse), bfloat16 dO ~ N(0,1); float32 dQ, dK, dV")
+BWD_CPU_N = 4096  # the oracle sample: the leading N x N causal block of one head
+
+
+def run_bwd(args, rank, world, local_rank):
+    """The backward pass of the 32K prefill: one fp8attn_bwd call (three launches) per step."""
+    import torch
+
+    from softmax_cast_precision_b200 import fp8attn
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+    w = WORKLOAD
+    q, k, v, _ = synthetic.workload_inputs(w, seed=rank_seed(rank))
+    do = synthetic.make_output_grad((w.B, w.H, w.N, w.d), rank_seed(rank) + 1)
+    qd, kd, vd = (torch.from_numpy(x).to(device) for x in (q, k, v))
+    dod = torch.from_numpy(do).to(device).to(torch.bfloat16)
+    del do
+    stream = torch.cuda.current_stream(device)
+    o, lse = fp8attn.fwd(qd, kd, vd, causal=w.causal, p_scale=P_SCALE, kv_order=KV_ORDER, stream=stream)
+
+    def step():
+        return fp8attn.bwd(qd, kd, vd, o, lse, dod, causal=w.causal, p_scale=P_SCALE, stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    fp8attn.check_error(stream=stream, device=device)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        torch.cuda.synchronize(device)
+        ev[0].record(stream)
+        for i in range(args.steps):
+            step()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+    fp8attn.check_error(stream=stream, device=device)
+    total_ms = max_over_ranks(ev[0].elapsed_time(ev[-1]), dist, device)
+    ms_per_step = total_ms / args.steps
+    pairs = w.B * w.H * w.N * (w.N + 1) // 2 if w.causal else w.B * w.H * w.N * w.N
+    flops = 10.0 * w.d * pairs  # five products of 2 d FLOPs per visible (query, key) pair
+    # End to end from pinned host buffers: the forward's inputs and outputs and dO in, the gradients out.
+    hosts = [t.cpu().pin_memory() for t in (qd, kd, vd, o, lse, dod)]
+    devs = [torch.empty_like(t) for t in (qd, kd, vd, o, lse, dod)]
+    outs = [torch.empty((w.B, w.H, w.N, w.d), dtype=torch.float32, pin_memory=True),
+            torch.empty((w.B, w.Hkv, w.N, w.d), dtype=torch.float32, pin_memory=True),
+            torch.empty((w.B, w.Hkv, w.N, w.d), dtype=torch.float32, pin_memory=True)]
+
+    def e2e_step():
+        for dst, src in zip(devs, hosts):
+            dst.copy_(src, non_blocking=True)
+        grads = fp8attn.bwd(*devs, causal=w.causal, p_scale=P_SCALE, stream=stream)
+        for dst, src in zip(outs, grads[:3]):
+            dst.copy_(src, non_blocking=True)
+
+    e2e_step()
+    barrier()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(3):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / 3, dist, device)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peak_bf16, _, peak_src = fp8_peak()
+    peak_bf16 /= FP8_OVER_BF16
+    # One product (S) at the FP8 rate, four (dP, dV, dK, dQ) at the 16-bit rate.
+    peak_mix = 1.0 / (0.8 / peak_bf16 + 0.2 / (peak_bf16 * FP8_OVER_BF16))
+    kernel_ms = statistics.mean(ev[i].elapsed_time(ev[i + 1]) for i in range(args.steps))
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    line = {
+        "metric": "FP8 P-cast attention backward TFLOP/s at N=32K, d=128", "unit": UNIT,
+        "value": aggregate_throughput(flops, world, ms_per_step), "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3 S / bf16 dP dV dK dQ", "data": "synthetic",
+        "config": {"workload": BWD_WORKLOAD_DESC, "flop_per_step_per_gpu": flops,
+                   "l2": "inputs exceed L2 (1.05 GB)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "gpu_launches": 3 * args.steps,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_mix, "unit": "TFLOP/s",
+                     "frac": achieved / peak_mix, "traffic": None,
+                     "peak_source": f"{peak_src}: one fifth of the FLOPs at x {FP8_OVER_BF16} (FP8/BF16 nominal) "
+                                    "of the bf16 cuBLAS burst rate, four fifths at it"},
+        "e2e": {"value": aggregate_throughput(flops, world, e2e_ms), "unit": UNIT,
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hosts),
+                "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in outs), "ms_per_step": e2e_ms},
+        "clocks": clk.summary(),
+    }
+    if not args.skip_cpu_baseline:
+        import oracle
+        from oracle import backward as Bw
+
+        n = BWD_CPU_N
+        qs, ks, vs = q[:1, :1, :n], k[:1, :1, :n], v[:1, :1, :n]
+        fwd_o = oracle.emulate(qs, ks, vs, causal=w.causal, block_n=128, p_scale=P_SCALE, reverse=bool(KV_ORDER))
+        dos = synthetic.make_output_grad((1, 1, n, w.d), 7)
+        t0 = time.perf_counter()
+        Bw.backward(qs, ks, vs, oracle.bf16_bits_to_float(fwd_o.o_bf16), fwd_o.lse, dos, causal=w.causal,
+                    p_scale=P_SCALE)
+        dt = time.perf_counter() - t0
+        f = 10.0 * w.d * (n * (n + 1) // 2 if w.causal else n * n)
+        from threadpoolctl import threadpool_info
+
+        blas = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+        line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": UNIT, "cores": max(blas) if blas else 1,
+                                "kind": "oracle",
+                                "sample": f"float64 backward oracle on the leading {n} x {n} block of one head "
+                                          f"({f / 1e12:.4f} TFLOP in {dt:.1f} s)"}
+    print(json.dumps(line), flush=True)
+
+
 def run_sharded(args, rank, world, local_rank):
     """Strong scaling: one 32K prefill split by kv heads across the ranks; a step
     is every rank's shard plus the all-gather of O and lse (NCCL)."""
@@ -814,13 +948,15 @@ def main():
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
-        if args.path in ("bf16qk", "decode"):
+        if args.path in ("bf16qk", "decode", "bwd"):
             raise SystemExit("--impl reference covers --path fp8 and wide")
         return run_reference_wide(args, rank) if args.path == "wide" else run_reference(args, rank, world)
     if args.shard == "heads":
         if args.path != "fp8" or args.impl != "ours":
             raise SystemExit("--shard heads covers the fp8 path")
         return run_sharded(args, rank, world, local_rank)
+    if args.path == "bwd":
+        return run_bwd(args, rank, world, local_rank)
     if args.path == "wide":
         return run_wide(args, rank, world, local_rank)
     if args.path == "bf16qk":
