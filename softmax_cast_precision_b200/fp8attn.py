@@ -159,6 +159,84 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_sc
     return o, lse
 
 
+def host_chunks(B: int, H: int, Hkv: int, N: int, chunks: int | None = None) -> list[tuple[int, int, int]]:
+    """The pieces ``fwd_host`` cuts a problem into: (b, kv head start, kv head end) triples, each within one
+    batch entry, covering every (batch, kv head) once, in order.  ``chunks`` is the target count (default:
+    about eight, fewer when a piece would hold under two waves of 148 persistent CTAs' work units); each
+    batch entry's kv heads are split into near-equal contiguous ranges."""
+    if B <= 0 or Hkv <= 0 or H % Hkv:
+        raise ValueError("need B >= 1, Hkv >= 1 and H a multiple of Hkv")
+    if chunks is None:
+        units = B * H * max(1, -(-N // 256))
+        chunks = max(1, min(8, units // (2 * 148)))
+    per_batch = max(1, min(Hkv, -(-int(chunks) // B)))
+    base, extra = divmod(Hkv, per_batch)
+    out = []
+    for b in range(B):
+        g0 = 0
+        for i in range(per_batch):
+            g1 = g0 + base + (1 if i < extra else 0)
+            out.append((b, g0, g1))
+            g0 = g1
+    return out
+
+
+def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_scale: float = 256.0,
+             kv_order="reverse", chunks: int | None = None, device=None):
+    """Forward pass of host tensors with the host<->device copies overlapped with the computation
+    (experimental: not yet run on a GPU).
+
+    q [B,H,N,d], k, v [B,Hkv,N,d] are E4M3 host tensors (pinned, for the copies to overlap).  The problem is
+    cut into pieces of whole kv heads with their query heads (``host_chunks``); piece c is copied to the device
+    on one stream, computed by ``fp8attn_fwd`` on a second once its copy is done, and copied back on a third,
+    so that the copies of one piece run during the computation of the others.  Returns pinned host (o, lse);
+    the call returns once both are complete.
+    """
+    q, k, v = _bytes(q), _bytes(k), _bytes(v)
+    B, H, Hkv, N, d = _shapes(q, k, v)
+    if q.is_cuda or k.is_cuda or v.is_cuda:
+        raise ValueError("fwd_host takes host tensors")
+    dev = torch.device(device if device is not None else "cuda:0")
+    rep = H // Hkv
+    o_h = torch.empty((B, H, N, d), dtype=torch.bfloat16, pin_memory=True)
+    lse_h = torch.empty((B, H, N), dtype=torch.float32, pin_memory=True)
+    if B * H * N == 0:
+        return o_h, lse_h
+    qd, kd, vd = (torch.empty(t.shape, dtype=torch.uint8, device=dev) for t in (q, k, v))
+    od = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    lsed = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    main = torch.cuda.current_stream(dev)
+    s_in, s_comp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+    for s in (s_in, s_comp, s_out):
+        s.wait_stream(main)  # the buffers above were allocated on the current stream
+    L = lib()
+    done = torch.cuda.Event()
+    for b, g0, g1 in host_chunks(B, H, Hkv, N, chunks):
+        h0, h1 = g0 * rep, g1 * rep
+        with torch.cuda.stream(s_in):
+            qd[b, h0:h1].copy_(q[b, h0:h1], non_blocking=True)
+            kd[b, g0:g1].copy_(k[b, g0:g1], non_blocking=True)
+            vd[b, g0:g1].copy_(v[b, g0:g1], non_blocking=True)
+        landed = torch.cuda.Event()
+        landed.record(s_in)
+        s_comp.wait_event(landed)
+        st = L.fp8attn_fwd(_ptr(qd[b, h0:h1]), _ptr(kd[b, g0:g1]), _ptr(vd[b, g0:g1]), _ptr(od[b, h0:h1]),
+                           _ptr(lsed[b, h0:h1]), 1, h1 - h0, g1 - g0, N, d, int(bool(causal)), ctypes.c_float(p_scale),
+                           _order(kv_order), ctypes.c_void_p(s_comp.cuda_stream))
+        if st != OK:
+            torch.cuda.synchronize(dev)
+            raise Fp8AttnError(st, "fp8attn_fwd")
+        computed = torch.cuda.Event()
+        computed.record(s_comp)
+        s_out.wait_event(computed)
+        with torch.cuda.stream(s_out):
+            o_h[b, h0:h1].copy_(od[b, h0:h1], non_blocking=True)
+            lse_h[b, h0:h1].copy_(lsed[b, h0:h1], non_blocking=True)
+    done.record(s_out)
+    done.synchronize()
+    return o_h, lse_h
+
+
 def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
                 lse_out: torch.Tensor | None = None, *, causal: bool, p_scale: float = 256.0,
                 kv_order="reverse", stream=None) -> None:
