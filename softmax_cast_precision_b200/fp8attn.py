@@ -132,30 +132,35 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_sc
     """
     q, k, v = _bytes(q), _bytes(k), _bytes(v)
     B, H, Hkv, N, d = _shapes(q, k, v)
-    host = not q.is_cuda
-    if host:
+    if not q.is_cuda:
+        # Host inputs: the copies in, the pass and the copies out all go on one stream (the given one, else
+        # the device's current stream), which the call waits for before returning.
         dev = torch.device(device if device is not None else "cuda:0")
-        q, k, v = (x.to(dev, non_blocking=True) for x in (q, k, v))
+        s = stream if stream is not None else torch.cuda.current_stream(dev)
+        with torch.cuda.stream(s):
+            qd, kd, vd = (x.to(dev, non_blocking=True) for x in (q, k, v))
+            o_d, lse_d = fwd(qd, kd, vd, causal=causal, p_scale=p_scale, kv_order=kv_order, with_lse=with_lse,
+                             stream=s)
+            o_h = out if out is not None else torch.empty(o_d.shape, dtype=o_d.dtype, pin_memory=True)
+            o_h.copy_(o_d, non_blocking=True)
+            lse_h = None
+            if lse_d is not None:
+                lse_h = lse_out if lse_out is not None else torch.empty(lse_d.shape, dtype=lse_d.dtype,
+                                                                        pin_memory=True)
+                lse_h.copy_(lse_d, non_blocking=True)
+        s.synchronize()
+        return o_h, lse_h
     dev = q.device
     if k.device != dev or v.device != dev:
         raise ValueError("q, k, v must be on the same device")
-    o = out if (out is not None and not host) else torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
+    o = out if out is not None else torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
     lse = None
     if with_lse:
-        lse = lse_out if (lse_out is not None and not host) else torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        lse = lse_out if lse_out is not None else torch.empty((B, H, N), dtype=torch.float32, device=dev)
     st = lib().fp8attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, N, d, int(bool(causal)),
                            ctypes.c_float(p_scale), _order(kv_order), _stream_ptr(dev, stream))
     if st != OK:
         raise Fp8AttnError(st, "fp8attn_fwd")
-    if host:
-        o_h = out if out is not None else torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        o_h.copy_(o, non_blocking=True)
-        lse_h = None
-        if lse is not None:
-            lse_h = lse_out if lse_out is not None else torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-            lse_h.copy_(lse, non_blocking=True)
-        torch.cuda.current_stream(dev).synchronize()
-        return o_h, lse_h
     return o, lse
 
 
