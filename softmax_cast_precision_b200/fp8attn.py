@@ -413,12 +413,16 @@ def fwd_scaled(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_scales: torc
 def fwd_wide(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_scale: float = 256.0,
              kv_order="reverse", signs=None, with_lse: bool = True, stream=None):
     """Attention on bfloat16/float32 q [B,H,N,d], k, v [B,Hkv,N,d]: quantise (Q, K per 128-row
-    block, V per head, rotated by ``signs`` when given), then the scaled forward pass."""
-    qc, qs = quantize(q, 128, signs, stream=stream)
-    kc, ks = quantize(k, 128, signs, stream=stream)
-    vc, vs = quantize(v, 0, signs, stream=stream)
-    return fwd_scaled(qc, kc, vc, qs, ks, vs, causal=causal, p_scale=p_scale, kv_order=kv_order, signs=signs,
-                      with_lse=with_lse, stream=stream)
+    block, V per head, rotated by ``signs`` when given), then the scaled forward pass.
+
+    The intermediate codes and scales are allocated on ``stream`` (when given), the stream that
+    reads them, so the caching allocator cannot hand their memory out while the pass still runs."""
+    with torch.cuda.stream(stream):
+        qc, qs = quantize(q, 128, signs, stream=stream)
+        kc, ks = quantize(k, 128, signs, stream=stream)
+        vc, vs = quantize(v, 0, signs, stream=stream)
+        return fwd_scaled(qc, kc, vc, qs, ks, vs, causal=causal, p_scale=p_scale, kv_order=kv_order,
+                          signs=signs, with_lse=with_lse, stream=stream)
 
 
 def pzero_count(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_scale: float = 256.0,
