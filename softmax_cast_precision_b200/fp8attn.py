@@ -309,12 +309,13 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, p_scale: float 
     if not q.is_cuda:
         raise ValueError("decode takes device tensors")
     need = int(lib().fp8attn_decode_workspace_bytes(B, H, N, int(split_tiles)))
-    ws = workspace if workspace is not None else torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    o = torch.empty((B, H, d), dtype=torch.bfloat16, device=q.device)
-    lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if with_lse else None
-    st = lib().fp8attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(),
-                              B, H, Hkv, N, d, ctypes.c_float(p_scale), _order(kv_order), int(split_tiles),
-                              _stream_ptr(q.device, stream))
+    with torch.cuda.stream(stream):  # a workspace made here is allocated on the stream that uses it
+        ws = workspace if workspace is not None else torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+        o = torch.empty((B, H, d), dtype=torch.bfloat16, device=q.device)
+        lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if with_lse else None
+        st = lib().fp8attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(ws),
+                                  ws.numel() * ws.element_size(), B, H, Hkv, N, d, ctypes.c_float(p_scale),
+                                  _order(kv_order), int(split_tiles), _stream_ptr(q.device, stream))
     if st != OK:
         raise Fp8AttnError(st, "fp8attn_decode")
     return o, lse
