@@ -1,4 +1,4 @@
-"""Oracle for the backward pass of the P-cast attention (groundwork: no kernel yet).
+"""Oracle for the backward pass of the P-cast attention (the reference of fp8attn_bwd).
 
 TEST INFRASTRUCTURE ONLY (like the rest of ``oracle``).
 

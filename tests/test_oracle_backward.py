@@ -1,5 +1,5 @@
-"""Pins of the backward-pass oracle (oracle.backward), groundwork for the
-backward kernel:
+"""Pins of the backward-pass oracle (oracle.backward), the reference of the
+backward kernels (fp8attn_bwd):
 
   * without the cast it is the exact gradient of softmax attention: it must
     equal PyTorch's automatic differentiation in float64 (causal and not,
