@@ -99,6 +99,20 @@ struct DqLayout {
   static constexpr int SMEM_BYTES = OFF_BAR + 128 + 1024;
 };
 
+// Every swizzled tile starts on a 1024-byte boundary (the 128-byte swizzle
+// pattern repeats every 8 rows of 128 bytes and is keyed to address bits
+// 7..9), and each kernel fits the 227 KB a CTA may opt into.
+static_assert(DkdvLayout::OFF_VF % 1024 == 0 && DkdvLayout::OFF_VB % 1024 == 0 && DkdvLayout::OFF_Q % 1024 == 0 &&
+                  DkdvLayout::OFF_QB % 1024 == 0 && DkdvLayout::OFF_DO % 1024 == 0 &&
+                  DkdvLayout::OFF_PT % 1024 == 0 && DkdvLayout::OFF_DST % 1024 == 0,
+              "dK/dV tiles must be 1024-byte aligned");
+static_assert(DqLayout::OFF_DO % 1024 == 0 && DqLayout::OFF_K % 1024 == 0 && DqLayout::OFF_V % 1024 == 0 &&
+                  DqLayout::OFF_KB % 1024 == 0 && DqLayout::OFF_VB % 1024 == 0 && DqLayout::OFF_DS % 1024 == 0,
+              "dQ tiles must be 1024-byte aligned");
+static_assert(DkdvLayout::OFF_BAR % 8 == 0 && DqLayout::OFF_BAR % 8 == 0, "mbarriers are 8-byte aligned");
+static_assert(DkdvLayout::SMEM_BYTES <= 227 * 1024 && DqLayout::SMEM_BYTES <= 227 * 1024,
+              "shared memory beyond the per-CTA opt-in limit");
+
 // Instruction descriptor for kind::f16 with bfloat16 A and B and an FP32
 // accumulator, with the operand majors given (bit 15: A MN-major, bit 16: B
 // MN-major).
