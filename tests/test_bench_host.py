@@ -80,3 +80,17 @@ def test_peak_falls_back_without_the_measured_file(tmp_path, monkeypatch):
     f.write_text(json.dumps({"bf16_tflops": 1000.0, "bf16_tflops_sustained": 900.0}))
     monkeypatch.setattr(bench, "PEAKS_FILE", str(f))
     assert bench.fp8_peak() == (1000.0 * bench.FP8_OVER_BF16, 900.0 * bench.FP8_OVER_BF16, "measured")
+
+
+@pytest.mark.parametrize("argv,message", [
+    (["--impl", "reference", "--path", "bwd"], "--impl reference covers"),
+    (["--impl", "reference", "--path", "decode"], "--impl reference covers"),
+    (["--shard", "heads", "--path", "wide"], "--shard heads covers"),
+    (["--warmup", "2"], "--warmup must be >= 3"),
+])
+def test_dispatch_guards_exit_before_any_device_work(argv, message, monkeypatch):
+    monkeypatch.setattr("sys.argv", ["bench.py", *argv])
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    with pytest.raises(SystemExit) as exc:
+        bench.main()
+    assert message in str(exc.value)
