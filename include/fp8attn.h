@@ -179,8 +179,7 @@ int fp8attn_decode(const void* q, const void* k, const void* v, void* o, float* 
 unsigned long long fp8attn_decode_workspace_bytes(int B, int H, int N, int split_tiles);
 
 /*
- * Backward pass of fp8attn_fwd (experimental: its GPU parity tests against
- * the oracle are pending).  Given the forward inputs q, k, v (E4M3), its
+ * Backward pass of fp8attn_fwd.  Given the forward inputs q, k, v (E4M3), its
  * outputs o (bfloat16 [B, H, N, d]) and lse (float32 [B, H, N], natural log,
  * as fp8attn_fwd writes it) and the output gradient dout (bfloat16 [B, H, N,
  * d]), writes the float32 gradients

@@ -188,8 +188,7 @@ def host_chunks(B: int, H: int, Hkv: int, N: int, chunks: int | None = None) -> 
 
 def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_scale: float = 256.0,
              kv_order="reverse", chunks: int | None = None, device=None):
-    """Forward pass of host tensors with the host<->device copies overlapped with the computation
-    (experimental: not yet run on a GPU).
+    """Forward pass of host tensors with the host<->device copies overlapped with the computation.
 
     q [B,H,N,d], k, v [B,Hkv,N,d] are E4M3 host tensors (pinned, for the copies to overlap).  The problem is
     cut into pieces of whole kv heads with their query heads (``host_chunks``); piece c is copied to the device
@@ -323,7 +322,7 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, p_scale: float 
 
 def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse: torch.Tensor,
         dout: torch.Tensor, *, causal: bool, p_scale: float = 256.0, stream=None):
-    """Backward pass of ``fwd`` (experimental; see fp8attn_bwd): gradients of the P-cast attention.
+    """Backward pass of ``fwd`` (see fp8attn_bwd): gradients of the P-cast attention.
 
     q, k, v are the forward's E4M3 inputs, o (bfloat16 [B,H,N,d]) and lse
     (float32 [B,H,N]) its outputs, dout the bfloat16 output gradient; all on

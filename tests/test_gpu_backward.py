@@ -21,11 +21,7 @@ from oracle import backward as Bw
 import synthetic
 from backward_bounds import error_bounds, violations
 
-pytestmark = [
-    pytest.mark.gpu,
-    pytest.mark.skip(reason="the backward kernels have not yet run on a GPU; these parity tests are enabled "
-                            "with their first run"),
-]
+pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")

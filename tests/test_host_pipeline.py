@@ -2,7 +2,7 @@
 
 CPU: the piece planner covers every (batch, kv head) exactly once, in order,
 in near-equal contiguous ranges that never cross a batch entry.
-GPU (skipped until the call first runs on a GPU): its outputs equal those of
+GPU: its outputs equal those of
 ``fwd`` on the same inputs bit for bit, since every (batch, head) slab is
 computed by the same kernel whatever the piece it belongs to.
 """
@@ -40,7 +40,6 @@ def test_host_chunks_rejects_bad_shapes():
 
 
 @pytest.mark.gpu
-@pytest.mark.skip(reason="fwd_host has not yet run on a GPU; enabled with its first run")
 @pytest.mark.parametrize("B,H,Hkv,N,chunks", [(1, 8, 8, 1000, 3), (2, 4, 2, 300, None), (1, 4, 4, 64, 1)])
 def test_fwd_host_equals_fwd(B, H, Hkv, N, chunks):
     from softmax_cast_precision_b200 import build
