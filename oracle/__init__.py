@@ -62,6 +62,7 @@ def _load():
         lib.oracle_e4m3_encode.argtypes = [ctypes.c_double]
         lib.oracle_e4m3_encode.restype = ctypes.c_uint8
         lib.oracle_e4m3_encode_array.argtypes = [P, P, i64]
+        lib.oracle_e4m3_encode_array_f64.argtypes = [P, P, i64]
         lib.oracle_e4m3_decode_array.argtypes = [P, P, i64]
         lib.oracle_bf16_round_array.argtypes = [P, P, i64]
         lib.oracle_attention_fp64.argtypes = [P, P, P, i32, i32, i32, i32, i32, i32, P, i32, P, P]
@@ -98,6 +99,14 @@ def e4m3_encode(x) -> np.ndarray:
     a = np.ascontiguousarray(x, dtype=np.float32)
     out = np.empty(a.shape, dtype=np.uint8)
     _load().oracle_e4m3_encode_array(_ptr(a), _ptr(out), a.size)
+    return out
+
+
+def e4m3_encode_f64(x) -> np.ndarray:
+    """Round float64 values to E4M3 bytes directly (same rule as ``e4m3_encode``)."""
+    a = np.ascontiguousarray(x, dtype=np.float64)
+    out = np.empty(a.shape, dtype=np.uint8)
+    _load().oracle_e4m3_encode_array_f64(_ptr(a), _ptr(out), a.size)
     return out
 
 

@@ -103,6 +103,13 @@ void oracle_e4m3_encode_array(const float* x, uint8_t* out, int64_t n)
         out[i] = oracle_e4m3_encode((double)x[i]);
 }
 
+/* The same rounding of float64 values (no intermediate float32 rounding). */
+void oracle_e4m3_encode_array_f64(const double* x, uint8_t* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = oracle_e4m3_encode(x[i]);
+}
+
 void oracle_e4m3_decode_array(const uint8_t* c, float* out, int64_t n)
 {
     for (int64_t i = 0; i < n; ++i)

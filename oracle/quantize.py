@@ -25,18 +25,19 @@ Readings taken where the page is silent (each is stated where it is used):
     query and key tiles of the forward kernel -- and V per (batch, head),
     because a per-tile V scale could not be divided out of the accumulated
     P V products.
-  * The rotation and the cast decision are taken in float32, the kernel's
-    precision: the rotation is evaluated as the radix-2 fast Walsh-Hadamard
-    transform with stages of half-width 1, 2, 4, ..., d/2 (pairs i and
-    i + h, sum first), then multiplied by float32(1 / sqrt(d)).  Its fp64
-    matrix definition is ``rotate_fp64`` and the two are pinned against each
-    other in the tests.
+  * The rotation is taken from its definition, x R as a float64 matrix
+    product (``rotate_fp64``), and the block maxima, descales and casts are
+    decided on those float64 values.  An implementation that evaluates R in
+    float32 (any fast transform) lands within a bounded distance of them, so
+    a comparison with it has to allow the neighbouring code exactly where a
+    float64 value lies within that bound of a rounding boundary; the tests
+    derive the bound and count those elements.
 """
 from __future__ import annotations
 
 import numpy as np
 
-from . import e4m3_decode, e4m3_encode
+from . import e4m3_decode, e4m3_encode_f64
 
 E4M3_MAX = 448.0
 
@@ -74,46 +75,6 @@ def unrotate_fp64(y, signs) -> np.ndarray:
     return (y @ hadamard_fp64(d) / np.sqrt(d)) * s
 
 
-def fwht_f32(x) -> np.ndarray:
-    """Unnormalised Walsh-Hadamard transform x H_d along the last axis, in float32.
-
-    Radix-2 stages of half-width h = 1, 2, ..., d/2; each stage maps the pair
-    (a, b) = (x[i], x[i + h]) with bit h of i clear to (a + b, a - b), every
-    sum and difference rounded to float32.
-    """
-    y = np.array(x, dtype=np.float32, copy=True)
-    d = y.shape[-1]
-    if d < 1 or d & (d - 1):
-        raise ValueError("d must be a power of two")
-    lead = y.shape[:-1]
-    h = 1
-    while h < d:
-        z = y.reshape(*lead, d // (2 * h), 2, h)
-        a = z[..., 0, :].copy()
-        b = z[..., 1, :]
-        z[..., 0, :] = a + b
-        z[..., 1, :] = a - b
-        y = z.reshape(*lead, d)
-        h *= 2
-    return y
-
-
-def rotate_f32(x, signs) -> np.ndarray:
-    """x R in float32: signs applied (exact), the transform, then one multiply by float32(1/sqrt(d))."""
-    x = np.asarray(x, dtype=np.float32)
-    d = x.shape[-1]
-    s = _check_signs(signs, d)
-    return fwht_f32(x * s) * np.float32(1.0 / np.sqrt(d))
-
-
-def unrotate_f32(y, signs) -> np.ndarray:
-    """y R^T in float32: the transform, one multiply by float32(1/sqrt(d)), then the signs."""
-    y = np.asarray(y, dtype=np.float32)
-    d = y.shape[-1]
-    s = _check_signs(signs, d)
-    return (fwht_f32(y) * np.float32(1.0 / np.sqrt(d))) * s
-
-
 def block_scale(amax) -> np.ndarray:
     """Smallest power of two s >= 2^-126 with amax <= 448 s (1 where amax is 0), as float32.
 
@@ -134,18 +95,20 @@ def block_scale(amax) -> np.ndarray:
 def quantize_blocks(x, block_rows: int, signs=None):
     """Cast [Z, N, d] values to E4M3 codes with one power-of-two scale per block of rows.
 
-    x is taken in float32 (bfloat16 inputs are exact in float32).  When
-    ``signs`` is given each row is rotated first (``rotate_f32``).  Blocks are
-    ``block_rows`` consecutive rows of one slab z (the last one ragged);
-    ``block_rows = 0`` means one block per slab.  Returns (codes uint8
+    x is taken as float32 values (bfloat16 inputs are exact in float32) and
+    carried in float64.  When ``signs`` is given each row is rotated first,
+    by the definition (``rotate_fp64``).  Blocks are ``block_rows``
+    consecutive rows of one slab z (the last one ragged); ``block_rows = 0``
+    means one block per slab.  A block's maximum, its descale and every
+    code are decided on the float64 values.  Returns (codes uint8
     [Z, N, d], scales float32 [Z, nblocks]) with x_rot ~= decode(codes) * scale.
     """
-    x = np.asarray(x, dtype=np.float32)
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
     if x.ndim != 3:
         raise ValueError("x must be [Z, N, d]")
     Z, N, d = x.shape
     if signs is not None:
-        x = rotate_f32(x, signs)
+        x = rotate_fp64(x, signs)
     br = N if block_rows == 0 else int(block_rows)
     if br <= 0:
         raise ValueError("block_rows must be >= 0")
@@ -159,7 +122,7 @@ def quantize_blocks(x, block_rows: int, signs=None):
         amax = np.abs(blk).reshape(Z, -1).max(axis=1)
         s = block_scale(amax)
         scales[:, b] = s
-        codes[:, b * br:(b + 1) * br, :] = e4m3_encode(blk / s[:, None, None])
+        codes[:, b * br:(b + 1) * br, :] = e4m3_encode_f64(blk / s.astype(np.float64)[:, None, None])
     return codes, scales
 
 
@@ -180,7 +143,8 @@ def quantized_attention(q, k, v, signs, *, causal: bool, p_scale: float, reverse
     given; cast Q and K with a scale per 128-row block and V with a scale per
     (batch, head); run the blockwise P-cast attention of the emulator on the
     dequantised values (exact: the scales are powers of two); rotate the
-    float32 output back by R^T and round it to bfloat16.  Returns a dict with
+    output back by R^T (float64 definition) and round it to bfloat16
+    (through float32).  Returns a dict with
     o (float32 values of the bfloat16 output, [B,H,R,d]), lse, the emulator
     result in the rotated frame and the codes and scales of Q, K and V.
     """
@@ -199,7 +163,7 @@ def quantized_attention(q, k, v, signs, *, causal: bool, p_scale: float, reverse
     vd = dequantize_blocks(vc, vs, 0).reshape(B, Hkv, N, d)
     res = emulate(qd, kd, vd, causal=causal, block_n=block_n, p_scale=p_scale, reverse=reverse,
                   n_sink=n_sink, rows=rows)
-    o32 = res.o_f32 if signs is None else unrotate_f32(res.o_f32, signs)
+    o32 = res.o_f32 if signs is None else unrotate_fp64(res.o_f32, signs).astype(np.float32)
     o = bf16_bits_to_float(bf16_round_bits(o32))
     return {"o": o, "lse": res.lse, "rotated": res,
             "q": (qc.reshape(B, H, N, d), qs), "k": (kc.reshape(B, Hkv, N, d), ks),

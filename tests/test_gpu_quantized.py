@@ -1,8 +1,13 @@
 """GPU parity of the quantisation path (fp8attn_quantize, fp8attn_fwd_scaled)
 against the oracle (oracle.quantize), through the C ABI.
 
-  * Codes and descales are integer/power-of-two decisions taken in float32 on
-    both sides in the same operation order, so they must match bit for bit.
+  * Codes and descales: without the rotation both sides cast the same
+    float32 values, so they match bit for bit.  With it, the oracle rotates by
+    the float64 definition and the kernel by a float32 fast transform; every
+    descale and code must then equal the oracle's except where the float64
+    value lies within the float32 transform's error bound of a rounding
+    boundary, where the neighbour is allowed too (tests/quant_bounds.py; the
+    number of such elements is reported and must be rare).
   * The scaled forward pass is compared like the plain one: per element
     max|O_gpu - O_oracle| <= 1e-2 * max|V|, lse within 1e-3.
   * Rotation with outlier channels lowers the error against exact attention
@@ -16,6 +21,7 @@ import torch
 import oracle
 from oracle import quantize as Qz
 import synthetic
+from quant_bounds import compare_codes
 
 pytestmark = pytest.mark.gpu
 
@@ -49,10 +55,15 @@ def test_quantize_bit_exact(fp8, d, dtype, block_rows, rotate):
     signs = synthetic.hadamard_signs(d, 21) if rotate else None
     codes, scales = fp8.quantize(_dev(x, dtype), block_rows, signs)
     torch.cuda.synchronize()
-    c_ref, s_ref = Qz.quantize_blocks(x, block_rows, signs)
-    assert np.array_equal(scales.cpu().numpy(), s_ref)
-    got = codes.cpu().numpy()
-    assert np.array_equal(got, c_ref), f"{(got != c_ref).sum()} codes differ"
+    got, s_got = codes.cpu().numpy(), scales.cpu().numpy()
+    if not rotate:
+        c_ref, s_ref = Qz.quantize_blocks(x, block_rows, None)
+        assert np.array_equal(s_got, s_ref)
+        assert np.array_equal(got, c_ref), f"{(got != c_ref).sum()} codes differ"
+    amb, amb_blk, bad_codes, bad_scales = compare_codes(x, block_rows, signs, got, s_got)
+    assert bad_scales == 0, f"{bad_scales} descales outside the allowance"
+    assert bad_codes == 0, f"{bad_codes} codes outside the allowance ({amb} ambiguous)"
+    assert amb <= 1e-3 * x.size, f"{amb} ambiguous elements"
 
 
 def test_quantize_empty_and_tiny(fp8):
