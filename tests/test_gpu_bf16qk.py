@@ -92,3 +92,34 @@ def test_kernel_faithful_scale_sweep(fp8):
     # with S = 256 (both at the quantisation-noise floor).
     assert mse["forward", 1.0] > 3.0 * mse["forward", 256.0]
     assert abs(mse["reverse", 256.0] - mse["forward", 256.0]) <= 0.05 * mse["forward", 256.0]
+
+
+def test_kernel_faithful_sawtooth_all_rows(fp8):
+    # The d_p sawtooth of the P-cast summary (section 2, condition 2) in
+    # measured GPU error: N = 4096, Delta = 7, reverse order (no collapse, so
+    # the cast's rounding is the error), every query row of 8 heads.  Powers
+    # of two share d_p = 2^-4 and give the same error; 96, 192 and 384 (d_p =
+    # 1.33 x 2^-4) and 320 (1.6 x 2^-4) are higher, and 448 (1.14 x 2^-4) sits
+    # between.  Per S the GPU's MSE against exact attention is within 5% of
+    # the emulator's, and the GPU's ratios to S = 256 follow the emulator's
+    # within 0.02, which with the pattern below reproduces the ordering.
+    N, H = 4096, 8
+    q, k, v8 = _inputs(1, H, H, N, 7.0, seed=91)
+    o64, _ = oracle.attention_fp64(q, k, v8, causal=False)
+    scales = (64.0, 96.0, 128.0, 192.0, 256.0, 320.0, 384.0, 448.0)
+    gpu, emu = {}, {}
+    for S in scales:
+        o, _ = _run(fp8, q, k, v8, False, S, "reverse")
+        ref = oracle.emulate(q, k, v8, causal=False, block_n=128, p_scale=S, reverse=True)
+        gpu[S] = float(np.mean((o - o64) ** 2))
+        emu[S] = float(np.mean((ref.o.astype(np.float64) - o64) ** 2))
+        assert abs(gpu[S] - emu[S]) <= 0.05 * emu[S], (S, gpu[S], emu[S])
+    r_gpu = {S: gpu[S] / gpu[256.0] for S in scales}
+    r_emu = {S: emu[S] / emu[256.0] for S in scales}
+    for S in scales:
+        assert abs(r_gpu[S] - r_emu[S]) <= 0.02, (S, r_gpu, r_emu)
+    for S in (64.0, 128.0):
+        assert abs(r_gpu[S] - 1.0) <= 0.01, r_gpu
+    for S in (96.0, 192.0, 320.0, 384.0):
+        assert r_gpu[S] >= 1.08, r_gpu
+    assert 1.03 <= r_gpu[448.0] < min(r_gpu[S] for S in (96.0, 192.0, 320.0, 384.0)), r_gpu
