@@ -252,6 +252,20 @@ const char* fp8attn_status_str(int status);
  */
 int fp8attn_check_error(void* stream);
 
+/*
+ * Test switch for the bounded waits (the pages have no counterpart).  Arms
+ * the next launch of the d = 128 forward kernel in this process
+ * (fp8attn_fwd, fp8attn_pzero_count, fp8attn_fwd_scaled, fp8attn_fwd_bf16qk):
+ * its producer skips the load of the first K tile, so the waits for that tile
+ * run out after wait_limit_ns nanoseconds instead of the normal 2 s.  The
+ * kernel then stops every role, lets its in-flight copies and products land,
+ * releases its tensor memory and returns; outputs of that launch are
+ * undefined and fp8attn_check_error() returns FP8ATTN_ERR_TIMEOUT.  Nothing
+ * faults or traps.  The switch is consumed by that one launch.  Returns
+ * FP8ATTN_ERR_INVALID_ARG unless 0 < wait_limit_ns <= 2e9.
+ */
+int fp8attn_test_withhold_load(unsigned long long wait_limit_ns);
+
 /* Library version as an integer (major * 10000 + minor * 100 + patch). */
 int fp8attn_version(void);
 

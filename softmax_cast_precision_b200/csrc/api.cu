@@ -12,6 +12,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/fp8attn.h"
@@ -32,6 +33,15 @@ __device__ uint32_t g_error_word;
 static __device__ __align__(256) unsigned int g_noalloc_scratch[FP8ATTN_NOALLOC_SCRATCH_BYTES / sizeof(unsigned int)];
 
 namespace {
+
+// How long a device-side wait of the persistent kernel may last before it
+// gives up and reports FP8ATTN_ERR_TIMEOUT.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+// Test switch (fp8attn_test_withhold_load): when non-zero, the next launch
+// of the persistent kernel skips its first K tile load and waits at most
+// this many nanoseconds.
+std::atomic<unsigned long long> g_test_withhold_ns{0};
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -174,6 +184,11 @@ int launch_v2(const void* q, const void* k, const void* v, FwdParams p, cudaStre
   p.num_q_tiles = (p.N + 127) / 128;
   p.num_kv_tiles = (p.N + 127) / 128;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
+  const unsigned long long withhold = g_test_withhold_ns.exchange(0ull);
+  if (withhold != 0ull) {
+    p.wait_limit_ns = withhold;
+    p.test_withhold_k = 1;
+  }
   const int num_pairs = (p.N + 255) / 256;
   const int64_t units = static_cast<int64_t>(p.B) * p.H * num_pairs;
   const int grid = static_cast<int>(units < sms ? units : sms);
@@ -235,6 +250,7 @@ FwdParams base_params(int B, int H, int Hkv, int N, int causal, float p_scale, i
   p.reverse = kv_order;
   p.p_scale = p_scale;
   p.log2_p_scale = static_cast<float>(std::log2(static_cast<double>(p_scale)));
+  p.wait_limit_ns = kWaitLimitNs;
   return p;
 }
 
@@ -594,6 +610,12 @@ extern "C" int fp8attn_check_error(void* stream) {
     if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return FP8ATTN_ERR_CUDA;
     return FP8ATTN_ERR_TIMEOUT;
   }
+  return FP8ATTN_OK;
+}
+
+extern "C" int fp8attn_test_withhold_load(unsigned long long wait_limit_ns) {
+  if (wait_limit_ns == 0ull || wait_limit_ns > kWaitLimitNs) return FP8ATTN_ERR_INVALID_ARG;
+  g_test_withhold_ns.store(wait_limit_ns);
   return FP8ATTN_OK;
 }
 

@@ -44,6 +44,11 @@ struct FwdParams {
   const float* v_scales;        // [B * Hkv]
   int unrotate;                 // rotate each output row back by R^T = H_D diag(signs) / sqrt(D)
   uint32_t sign_bits[4];        // bit i set: signs[i] = -1
+  // Persistent kernel: how long a wait may last before it gives up (2 s in
+  // normal use), and the test switch that makes the producer skip the load
+  // of the first K tile, so that a wait runs out on purpose.
+  unsigned long long wait_limit_ns;
+  int test_withhold_k;
 };
 
 template <int D>

@@ -79,6 +79,7 @@ struct V2Bars {
   // hands them to the other roles through a two-slot queue.
   uint64_t unit_full[2], unit_empty[2];
   int unit_id[2];
+  uint64_t wait_limit_ns;  // bound of every wait (FwdParams::wait_limit_ns)
   uint32_t tmem_base;
   volatile uint32_t abort;
 };
@@ -136,7 +137,8 @@ __device__ __forceinline__ int stream_tile(const FwdParams& p, const UnitGeom& g
   return p.reverse ? (g.ntiles - 1 - idx) : idx;
 }
 
-// Wait with a time limit; also gives up as soon as another role aborted.
+// Wait with a time limit (bars->wait_limit_ns); also gives up as soon as
+// another role aborted.
 // Between checks the thread sleeps inside try_wait (suspend hint), so a
 // waiting warp takes no issue slots from the warps sharing its scheduler and
 // still wakes as soon as the phase completes.
@@ -147,7 +149,7 @@ __device__ __forceinline__ bool v2_wait(V2Bars* bars, uint64_t* bar, uint32_t pa
   while (true) {
     if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (bars->abort) return false;
-    if (globaltimer_ns() - t0 > 2000000000ull) {
+    if (globaltimer_ns() - t0 > bars->wait_limit_ns) {
       atomicOr(err_word, code);
       bars->abort = 1u;
       return false;
@@ -225,6 +227,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
       mbar_init(&bars->unit_empty[s2], kUnitReaders);
     }
     bars->abort = 0u;
+    bars->wait_limit_ns = p.wait_limit_ns;
     fence_mbar_init();
   }
   if (warp == 9) {
@@ -284,7 +287,9 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
             ok = v2_wait(bars, &bars->k_free[st], ((kv_it / L::STAGES) - 1) & 1, err_word, kErrTimeoutPipe);
             if (!ok) break;
           }
-          load_qk(base + L::OFF_K + st * L::QK_TILE, &tm_k, &bars->k_full[st], t * 128, g.zkv);
+          // (The test switch skips the first K tile: its readers' waits run out.)
+          if (!(p.test_withhold_k && kv_it == 0))
+            load_qk(base + L::OFF_K + st * L::QK_TILE, &tm_k, &bars->k_full[st], t * 128, g.zkv);
           if (kv_it >= L::STAGES) {
             ok = v2_wait(bars, &bars->v_free[st], ((kv_it / L::STAGES) - 1) & 1, err_word, kErrTimeoutPipe);
             if (!ok) break;
@@ -300,7 +305,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         if (q_done[0] > 0) drain_wait(&bars->q_full[0], (q_done[0] - 1) & 1);
         if (q_done[1] > 0) drain_wait(&bars->q_full[1], (q_done[1] - 1) & 1);
         for (uint32_t i = (kv_it > L::STAGES ? kv_it - L::STAGES : 0); i < kv_it; ++i) {
-          drain_wait(&bars->k_full[i % L::STAGES], (i / L::STAGES) & 1);
+          if (!(p.test_withhold_k && i == 0)) drain_wait(&bars->k_full[i % L::STAGES], (i / L::STAGES) & 1);
           drain_wait(&bars->v_full[i % L::STAGES], (i / L::STAGES) & 1);
         }
       }

@@ -245,3 +245,9 @@ def test_bwd_binding_checks(fp8):
         fp8.bwd(u8, u8, u8, b16, lse, b16, causal=True)  # host tensors
     with pytest.raises(ValueError):
         fp8.bwd(u8, u8[:, :, :4], u8, b16, lse, b16, causal=True)  # k disagrees on N
+
+
+def test_withhold_switch_validation(fp8):
+    L = fp8.lib()
+    assert L.fp8attn_test_withhold_load(0) == fp8.ERR_INVALID_ARG
+    assert L.fp8attn_test_withhold_load(2_000_000_001) == fp8.ERR_INVALID_ARG
