@@ -32,6 +32,7 @@ forward's inputs, O, lse and a bfloat16 dO).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import re
 import json
@@ -81,6 +82,9 @@ def parse_args():
                          "split one problem's kv heads and all-gather the output (strong scaling)")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (used under ncu)")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="run the fp8 path's prefill at this sequence length instead of 32768 (a smaller case "
+                         "for profiling; not the headline workload)")
     return ap.parse_args()
 
 
@@ -114,6 +118,15 @@ def kernel_source_hash() -> str:
     m = re.search(r"\nint launch_v2\(.*?\n}\n", api, re.S)
     h.update(_strip_comments(m.group(0) if m else api).encode())
     return h.hexdigest()[:16]
+
+
+def peak_clock_mhz():
+    """Median SM clock under load while the measured peaks were taken (None if unknown)."""
+    try:
+        with open(PEAKS_FILE) as fh:
+            return float(json.load(fh)["clocks_under_load"]["sm_mhz_median"])
+    except (OSError, KeyError, ValueError, TypeError):
+        return None
 
 
 def fp8_peak():
@@ -940,6 +953,24 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def set_seq_len(args):
+    """A smaller case of the same workload for profiling (--seq-len): the
+    prefill paths run at sequence length N, the decode path against N keys."""
+    global WORKLOAD, WORKLOAD_DESC, WIDE_WORKLOAD_DESC, BF16QK_WORKLOAD_DESC, BWD_WORKLOAD_DESC
+    n = args.seq_len
+    if args.impl != "ours" or args.shard != "replicas" or n < 1:
+        raise SystemExit("--seq-len covers our implementation with replicas")
+    if args.path == "decode":
+        DECODE_SHAPE["N"] = n
+        return
+    WORKLOAD = dataclasses.replace(WORKLOAD, name=f"prefill{n}", N=n)
+    tag = f"N={n} (profiling case, not the headline)"
+    WORKLOAD_DESC = WORKLOAD_DESC.replace("N=32768", tag)
+    WIDE_WORKLOAD_DESC = WIDE_WORKLOAD_DESC.replace("N=32768", tag)
+    BF16QK_WORKLOAD_DESC = BF16QK_WORKLOAD_DESC.replace("N=32768", tag)
+    BWD_WORKLOAD_DESC = BWD_WORKLOAD_DESC.replace("N=32768", tag)
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -947,6 +978,8 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.seq_len is not None:
+        set_seq_len(args)
     if args.impl == "reference":
         if args.path in ("bf16qk", "decode", "bwd"):
             raise SystemExit("--impl reference covers --path fp8 and wide")
@@ -1016,22 +1049,30 @@ def main():
     value = aggregate_throughput(flops, world, ms_per_step)
 
     # --- end to end through the public API with host buffers ----------------
+    # fwd_host: pinned host inputs and outputs, the copies in and out
+    # overlapped with the computation piece by piece; each call returns once
+    # the outputs are on the host, and its streams start after and join back
+    # into the current stream, so events on that stream span whole calls.
     qh, kh, vh = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
     oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
     e2e_steps = max(3, min(args.steps, 10))
-    fp8attn.fwd(qh, kh, vh, causal=w.causal, p_scale=P_SCALE, kv_order=KV_ORDER, out=oh, lse_out=lh,
-                device=device)
+
+    def e2e_step():
+        fp8attn.fwd_host(qh, kh, vh, causal=w.causal, p_scale=P_SCALE, kv_order=KV_ORDER, out=oh, lse_out=lh,
+                         device=device)
+
+    e2e_step()
     barrier()
     torch.cuda.synchronize(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        fp8attn.fwd(qh, kh, vh, causal=w.causal, p_scale=P_SCALE, kv_order=KV_ORDER, out=oh, lse_out=lh,
-                    device=device)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(device)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, device)
+    fp8attn.check_error(stream=stream, device=device)
     h2d = q.nbytes + k.nbytes + v.nbytes
     d2h = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
 
@@ -1045,7 +1086,12 @@ def main():
     peak_burst, peak_sustained, peak_src = fp8_peak()
     kernel_ms = statistics.mean(per_step)
     achieved = flops / (kernel_ms * 1e-3) / 1e12
-    traffic = traffic_per_launch()
+    traffic = traffic_per_launch() if args.seq_len is None else None
+    clocks = clk.summary()
+    # The measured peak was taken at its own (power-capped) clock; the same
+    # peak scaled to the clock this kernel ran at gives the fraction per clock.
+    p_mhz, k_mhz = peak_clock_mhz(), clocks.get("sm_mhz")
+    frac_clock = achieved / (peak_burst * k_mhz / p_mhz) if p_mhz and k_mhz else None
     line = {
         "metric": METRIC,
         "value": value,
@@ -1059,16 +1105,21 @@ def main():
         "vs_baseline": None,
         "dtype": "e4m3",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD_DESC, "flop_per_step_per_gpu": flops, "l2": "inputs exceed L2 (402 MB)",
+        "config": {"workload": WORKLOAD_DESC, "flop_per_step_per_gpu": flops,
+                   "l2": f"inputs exceed L2 ({(q.nbytes + k.nbytes + v.nbytes) / 1e6:.0f} MB)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "gpu_launches": args.steps,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_burst, "unit": "TFLOP/s",
                      "frac": achieved / peak_burst, "traffic": traffic,
                      "peak_source": f"{peak_src}: bf16 cuBLAS burst x {FP8_OVER_BF16} (FP8/BF16 nominal)",
-                     "frac_of_sustained": achieved / peak_sustained},
+                     "frac_of_sustained": achieved / peak_sustained,
+                     "frac_at_kernel_clock": frac_clock,
+                     "clock_note": (f"peak measured at a median {p_mhz} MHz, this kernel at {k_mhz} MHz: "
+                                    "frac_at_kernel_clock = achieved / (peak x kernel MHz / peak MHz)")},
         "e2e": {"value": aggregate_throughput(flops, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "clocks": clk.summary(),
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                "how": "fwd_host with pinned host buffers, copies overlapped piece by piece; CUDA events"},
+        "clocks": clocks,
         "mse_vs_fp64": {"value": mse, "rows": "256 evenly spaced query rows of each head",
                         "reference": "PyTorch float64 softmax(QK^T/sqrt(d))V on the same E4M3 inputs"},
     }

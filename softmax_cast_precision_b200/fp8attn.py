@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
         L.fp8attn_check_error.argtypes = [P]
         L.fp8attn_check_error.restype = i32
         L.fp8attn_version.restype = i32
+        L.fp8attn_test_withhold_load.argtypes = [u64]
+        L.fp8attn_test_withhold_load.restype = i32
         _lib = L
         return L
 
@@ -117,6 +119,12 @@ def _stream_ptr(device: torch.device, stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _on_device(device: torch.device):
+    """Make ``device`` current for a library call: the library takes its per-device state (SM count, pools,
+    scratch, error word) from the current device."""
+    return torch.cuda.device(device)
+
+
 def _ptr(t) -> ctypes.c_void_p:
     return ctypes.c_void_p(t.data_ptr() if t is not None and t.numel() else 0)
 
@@ -157,8 +165,9 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_sc
     lse = None
     if with_lse:
         lse = lse_out if lse_out is not None else torch.empty((B, H, N), dtype=torch.float32, device=dev)
-    st = lib().fp8attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, N, d, int(bool(causal)),
-                           ctypes.c_float(p_scale), _order(kv_order), _stream_ptr(dev, stream))
+    with _on_device(q.device):
+        st = lib().fp8attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, N, d, int(bool(causal)),
+                               ctypes.c_float(p_scale), _order(kv_order), _stream_ptr(dev, stream))
     if st != OK:
         raise Fp8AttnError(st, "fp8attn_fwd")
     return o, lse
@@ -187,14 +196,17 @@ def host_chunks(B: int, H: int, Hkv: int, N: int, chunks: int | None = None) -> 
 
 
 def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_scale: float = 256.0,
-             kv_order="reverse", chunks: int | None = None, device=None):
+             kv_order="reverse", chunks: int | None = None, device=None, out: torch.Tensor | None = None,
+             lse_out: torch.Tensor | None = None):
     """Forward pass of host tensors with the host<->device copies overlapped with the computation.
 
     q [B,H,N,d], k, v [B,Hkv,N,d] are E4M3 host tensors (pinned, for the copies to overlap).  The problem is
     cut into pieces of whole kv heads with their query heads (``host_chunks``); piece c is copied to the device
-    on one stream, computed by ``fp8attn_fwd`` on a second once its copy is done, and copied back on a third,
-    so that the copies of one piece run during the computation of the others.  Returns pinned host (o, lse);
-    the call returns once both are complete.
+    on one stream, computed by ``fp8attn_fwd`` once its copy is done, and copied back on a third stream, so that
+    the copies of one piece run during the computation of the others.  The pieces' passes alternate between two
+    streams, so that one piece's persistent kernel can start on the SMs the previous one has finished with.
+    Returns host (o, lse): ``out`` (bfloat16 [B,H,N,d]) and ``lse_out`` (float32 [B,H,N]) when given (pinned,
+    for the copies to overlap), else new pinned tensors.  The call returns once both are complete.
     """
     q, k, v = _bytes(q), _bytes(k), _bytes(v)
     B, H, Hkv, N, d = _shapes(q, k, v)
@@ -202,20 +214,37 @@ def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool,
         raise ValueError("fwd_host takes host tensors")
     dev = torch.device(device if device is not None else "cuda:0")
     rep = H // Hkv
-    o_h = torch.empty((B, H, N, d), dtype=torch.bfloat16, pin_memory=True)
-    lse_h = torch.empty((B, H, N), dtype=torch.float32, pin_memory=True)
+    o_h = out if out is not None else torch.empty((B, H, N, d), dtype=torch.bfloat16, pin_memory=True)
+    lse_h = lse_out if lse_out is not None else torch.empty((B, H, N), dtype=torch.float32, pin_memory=True)
+    if (o_h.is_cuda or lse_h.is_cuda or o_h.dtype != torch.bfloat16 or lse_h.dtype != torch.float32
+            or tuple(o_h.shape) != (B, H, N, d) or tuple(lse_h.shape) != (B, H, N)
+            or not o_h.is_contiguous() or not lse_h.is_contiguous()):
+        raise ValueError("out / lse_out must be contiguous host tensors: bfloat16 [B,H,N,d] and float32 [B,H,N]")
     if B * H * N == 0:
         return o_h, lse_h
     qd, kd, vd = (torch.empty(t.shape, dtype=torch.uint8, device=dev) for t in (q, k, v))
     od = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
     lsed = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     main = torch.cuda.current_stream(dev)
-    s_in, s_comp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
-    for s in (s_in, s_comp, s_out):
+    s_in, s_c0, s_c1, s_out = (torch.cuda.Stream(device=dev) for _ in range(4))
+    for s in (s_in, s_c0, s_c1, s_out):
         s.wait_stream(main)  # the buffers above were allocated on the current stream
     L = lib()
     done = torch.cuda.Event()
-    for b, g0, g1 in host_chunks(B, H, Hkv, N, chunks):
+    with _on_device(dev):
+        _fwd_host_pieces(L, q, k, v, qd, kd, vd, od, lsed, o_h, lse_h, B, H, Hkv, N, d, rep, causal, p_scale,
+                         kv_order, chunks, dev, s_in, s_c0, s_c1, s_out)
+    done.record(s_out)
+    main.wait_event(done)  # work ordered after this call on the current stream follows the copies out
+    done.synchronize()
+    return o_h, lse_h
+
+
+def _fwd_host_pieces(L, q, k, v, qd, kd, vd, od, lsed, o_h, lse_h, B, H, Hkv, N, d, rep, causal, p_scale, kv_order,
+                     chunks, dev, s_in, s_c0, s_c1, s_out):
+    """The piece loop of ``fwd_host``: copy in, compute (alternating s_c0 / s_c1), copy out."""
+    for c, (b, g0, g1) in enumerate(host_chunks(B, H, Hkv, N, chunks)):
+        s_comp = s_c1 if c & 1 else s_c0
         h0, h1 = g0 * rep, g1 * rep
         with torch.cuda.stream(s_in):
             qd[b, h0:h1].copy_(q[b, h0:h1], non_blocking=True)
@@ -236,9 +265,6 @@ def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool,
         with torch.cuda.stream(s_out):
             o_h[b, h0:h1].copy_(od[b, h0:h1], non_blocking=True)
             lse_h[b, h0:h1].copy_(lsed[b, h0:h1], non_blocking=True)
-    done.record(s_out)
-    done.synchronize()
-    return o_h, lse_h
 
 
 def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
@@ -266,9 +292,10 @@ def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Te
     if lse_out is not None and (lse_out.device != q.device or lse_out.dtype != torch.float32
                                 or tuple(lse_out.shape) != (B, H, N) or not lse_out.is_contiguous()):
         raise ValueError("lse_out must be a contiguous float32 [B,H,N] tensor on the inputs' device")
-    st = lib().fp8attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse_out), B, H, Hkv, N, d,
-                                   int(bool(causal)), ctypes.c_float(p_scale), _order(kv_order),
-                                   _stream_ptr(q.device, stream))
+    with _on_device(q.device):
+        st = lib().fp8attn_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse_out), B, H, Hkv, N, d,
+                                       int(bool(causal)), ctypes.c_float(p_scale), _order(kv_order),
+                                       _stream_ptr(q.device, stream))
     if st != OK:
         raise Fp8AttnError(st, "fp8attn_fwd_noalloc")
 
@@ -286,8 +313,9 @@ def fwd_bf16qk(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: boo
         raise ValueError("fwd_bf16qk takes device tensors")
     o = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q.device)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if with_lse else None
-    st = lib().fp8attn_fwd_bf16qk(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, N, d, int(bool(causal)),
-                                  ctypes.c_float(p_scale), _order(kv_order), _stream_ptr(q.device, stream))
+    with _on_device(q.device):
+        st = lib().fp8attn_fwd_bf16qk(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, H, Hkv, N, d, int(bool(causal)),
+                                      ctypes.c_float(p_scale), _order(kv_order), _stream_ptr(q.device, stream))
     if st != OK:
         raise Fp8AttnError(st, "fp8attn_fwd_bf16qk")
     return o, lse
@@ -343,9 +371,10 @@ def bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor, lse:
     dk = torch.empty((B, Hkv, N, d), **f32)
     dv = torch.empty((B, Hkv, N, d), **f32)
     delta = torch.empty((B, H, N), **f32)
-    st = lib().fp8attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
-                           _ptr(delta), B, H, Hkv, N, d, int(bool(causal)), ctypes.c_float(p_scale),
-                           _stream_ptr(q.device, stream))
+    with _on_device(q.device):
+        st = lib().fp8attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                               _ptr(delta), B, H, Hkv, N, d, int(bool(causal)), ctypes.c_float(p_scale),
+                               _stream_ptr(q.device, stream))
     if st != OK:
         raise Fp8AttnError(st, "fp8attn_bwd")
     return dq, dk, dv, delta
@@ -381,8 +410,9 @@ def quantize(x: torch.Tensor, block_rows: int, signs=None, *, out: torch.Tensor 
     codes = out if out is not None else torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     sc = scales if scales is not None else torch.empty((Z, nb), dtype=torch.float32, device=x.device)
     keep, sp = _host_signs(signs, d)
-    st = lib().fp8attn_quantize(_ptr(x), 0 if x.dtype == torch.bfloat16 else 1, _ptr(codes), _ptr(sc), Z, N, d,
-                                int(block_rows), sp, _stream_ptr(x.device, stream))
+    with _on_device(x.device):
+        st = lib().fp8attn_quantize(_ptr(x), 0 if x.dtype == torch.bfloat16 else 1, _ptr(codes), _ptr(sc), Z, N, d,
+                                    int(block_rows), sp, _stream_ptr(x.device, stream))
     del keep
     if st != OK:
         raise Fp8AttnError(st, "fp8attn_quantize")
@@ -401,9 +431,10 @@ def fwd_scaled(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_scales: torc
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if with_lse else None
     qs, ks, vs = (t.contiguous().float() for t in (q_scales, k_scales, v_scales))
     keep, sp = _host_signs(signs, d)
-    st = lib().fp8attn_fwd_scaled(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(qs), _ptr(ks), _ptr(vs), sp,
-                                  B, H, Hkv, N, d, int(bool(causal)), ctypes.c_float(p_scale), _order(kv_order),
-                                  _stream_ptr(q.device, stream))
+    with _on_device(q.device):
+        st = lib().fp8attn_fwd_scaled(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(qs), _ptr(ks), _ptr(vs), sp,
+                                      B, H, Hkv, N, d, int(bool(causal)), ctypes.c_float(p_scale), _order(kv_order),
+                                      _stream_ptr(q.device, stream))
     del keep
     if st != OK:
         raise Fp8AttnError(st, "fp8attn_fwd_scaled")
@@ -436,9 +467,10 @@ def pzero_count(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bo
     if not q.is_cuda:
         raise ValueError("pzero_count takes device tensors")
     counts = out if out is not None else torch.empty((B, H), dtype=torch.int64, device=q.device)
-    st = lib().fp8attn_pzero_count(_ptr(q), _ptr(k), _ptr(v), _ptr(counts), B, H, Hkv, N, d, int(bool(causal)),
-                                   ctypes.c_float(p_scale), _order(kv_order), int(n_sink),
-                                   _stream_ptr(q.device, stream))
+    with _on_device(q.device):
+        st = lib().fp8attn_pzero_count(_ptr(q), _ptr(k), _ptr(v), _ptr(counts), B, H, Hkv, N, d, int(bool(causal)),
+                                       ctypes.c_float(p_scale), _order(kv_order), int(n_sink),
+                                       _stream_ptr(q.device, stream))
     if st != OK:
         raise Fp8AttnError(st, "fp8attn_pzero_count")
     return counts
@@ -450,6 +482,14 @@ def check_error(stream=None, device=None) -> None:
     st = lib().fp8attn_check_error(_stream_ptr(dev, stream))
     if st != OK:
         raise Fp8AttnError(st, "fp8attn_check_error")
+
+
+def test_withhold_load(wait_limit_ns: int) -> None:
+    """Test switch: the next d = 128 forward launch skips its first K tile load and its waits give up after
+    ``wait_limit_ns`` (see fp8attn_test_withhold_load); check_error() then raises with ERR_TIMEOUT."""
+    st = lib().fp8attn_test_withhold_load(int(wait_limit_ns))
+    if st != OK:
+        raise Fp8AttnError(st, "fp8attn_test_withhold_load")
 
 
 def raw_call(name: str, *args) -> int:

@@ -87,6 +87,8 @@ def test_peak_falls_back_without_the_measured_file(tmp_path, monkeypatch):
     (["--impl", "reference", "--path", "decode"], "--impl reference covers"),
     (["--shard", "heads", "--path", "wide"], "--shard heads covers"),
     (["--warmup", "2"], "--warmup must be >= 3"),
+    (["--seq-len", "4096", "--impl", "reference"], "--seq-len covers"),
+    (["--seq-len", "4096", "--shard", "heads"], "--seq-len covers"),
 ])
 def test_dispatch_guards_exit_before_any_device_work(argv, message, monkeypatch):
     monkeypatch.setattr("sys.argv", ["bench.py", *argv])
@@ -94,3 +96,15 @@ def test_dispatch_guards_exit_before_any_device_work(argv, message, monkeypatch)
     with pytest.raises(SystemExit) as exc:
         bench.main()
     assert message in str(exc.value)
+
+
+def test_peak_clock_for_the_clock_normalised_fraction(tmp_path, monkeypatch):
+    f = tmp_path / "peaks.json"
+    f.write_text(json.dumps({"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0,
+                             "clocks_under_load": {"sm_mhz_median": 1312.0}}))
+    monkeypatch.setattr(bench, "PEAKS_FILE", str(f))
+    assert bench.peak_clock_mhz() == 1312.0
+    f.write_text(json.dumps({"bf16_tflops": 1600.0}))
+    assert bench.peak_clock_mhz() is None
+    monkeypatch.setattr(bench, "PEAKS_FILE", str(tmp_path / "missing.json"))
+    assert bench.peak_clock_mhz() is None
