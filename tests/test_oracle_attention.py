@@ -195,8 +195,13 @@ def test_paper_magnitudes_at_n4096():
     # forward S=1 is 3-10x worse than the optimised configurations
     for opt in (f256, r256):
         assert FACTS["mse_ratio_fwd1_low"] <= base / opt <= FACTS["mse_ratio_fwd1_high"]
-    # forward S=256 below forward S=448 (the pages say by 10-15%; this
-    # construction gives a smaller gap, see the design notes)
+    # forward S=256 below forward S=448.  The pages say by 10-15%; here the
+    # gap is 5-7%.  d_p(S) is the step met by the largest P values, just
+    # below the row maximum (at 448 it is 1.14x that at 256); the many
+    # smaller P values fall at positions in their E4M3 binades that do not
+    # favour either scale, so they add the same error to both and dilute
+    # the ratio.  The lower bound of 2% keeps the direction and the order
+    # of magnitude.
     assert f256 < f448
     assert 0.02 <= 1.0 - f256 / f448 <= FACTS["mse_gain_256_vs_448_high"]
     # saturation: reverse + 256 indistinguishable from forward + 256
