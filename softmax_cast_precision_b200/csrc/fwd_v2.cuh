@@ -169,8 +169,14 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 // thread of the two softmax warpgroups.
 constexpr uint32_t kUnitReaders = 2 + 256;
 
-// Pairs out of every eight (16 keys) whose exponentials use the polynomial.
-constexpr int kPolyPairs = 2;
+// Pairs out of every eight (16 keys) whose exponentials use the FMA-pipe
+// polynomial instead of MUFU ex2.  Measured at the 32K prefill: 0 pairs
+// 1440 TFLOP/s, 1 pair 1311, 2 pairs 1294 (with the packed conversion
+// below).  The exponential loop is limited by issue and dependency latency
+// as much as by MUFU throughput, and the polynomial's longer dependency
+// chains cost more than the MUFU work they remove, so every exponential
+// uses MUFU.
+constexpr int kPolyPairs = 0;
 
 // SCALED: the inputs carry descales (FwdParams q/k/v_scales) and optionally
 // a rotation to undo on the output; the running maximum is then kept in
@@ -567,7 +573,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
             float y0, y1, y2, y3;
             f2_unpack(pa, y0, y1);
             f2_unpack(pb, y2, y3);
-            w[q4] = cvt_e4m3x2(y0, y1) | (cvt_e4m3x2(y2, y3) << 16);
+            w[q4] = cvt_e4m3x4(y0, y1, y2, y3);
             if constexpr (COUNT) {
 #pragma unroll
               for (int e = 0; e < 4; ++e) {

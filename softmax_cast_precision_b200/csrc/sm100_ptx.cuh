@@ -252,6 +252,19 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   return static_cast<uint32_t>(r);
 }
 
+// Four FP32 values to four E4M3 bytes (a in bits 0..7), same rounding: the
+// two conversions write the halves of one 32-bit register directly.
+__device__ __forceinline__ uint32_t cvt_e4m3x4(float a, float b, float c, float e) {
+  uint32_t r;
+  asm("{\n\t.reg .b16 lo, hi;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
+      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
+      "mov.b32 %0, {lo, hi};\n\t}"
+      : "=r"(r)
+      : "f"(a), "f"(b), "f"(c), "f"(e));
+  return r;
+}
+
 // Packed FP32 pairs (sm_100 f32x2 arithmetic): one instruction, two lanes.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
   uint64_t r;
@@ -289,9 +302,11 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // in the low mantissa bits), f = x - j in [-1/2, 1/2], 2^f from a degree-4
 // minimax polynomial (coefficients fitted by gen_exp2_poly.py; relative error
 // 2.7e-6 in float32), and 2^j applied by adding j to the exponent field.
-// Arguments below -125 are clamped there (2^-125 is negligible next to the
-// row maximum's 2^log2(S) >= 2^-64 and casts to E4M3 zero), which also maps
-// -inf to a finite tiny value.
+// Arguments below -125 are clamped there, which also maps -inf (a masked
+// key) to 2^-125 instead of 0: it casts to E4M3 zero like 0 does, and added
+// to a row sum l * S >= S >= 2^-64 (the row maximum's own term) it leaves
+// that float32 sum unchanged (its ulp is at least 2^-87), so the result is
+// the same as for an exact 0.
 __device__ __forceinline__ uint64_t exp2_poly2(float x0, float x1) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
   const uint64_t x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
