@@ -513,11 +513,15 @@ extern "C" int fp8attn_decode(const void* q, const void* k, const void* v, void*
   p.reverse = kv_order;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
   p.log2_p_scale = static_cast<float>(std::log2(static_cast<double>(p_scale)));
-  constexpr int kSmem = 4 * 128 * 128 + 2 * kDecodeMaxG * 128 * 4 + 4 * kDecodeMaxG * 4;
-  if (cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
+  CUtensorMap tk, tv;
+  if (!make_map(&tk, k, 128, N, B * Hkv, 128) || !make_map(&tv, v, 128, N, B * Hkv, 128)) return FP8ATTN_ERR_CUDA;
+  uint32_t* err_word = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err_word), g_error_word) != cudaSuccess) return FP8ATTN_ERR_CUDA;
+  if (cudaFuncSetAttribute(decode_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, DecodeLayout::SMEM_BYTES) !=
+      cudaSuccess)
     return FP8ATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  decode_split_kernel<<<dim3(p.splits, B * Hkv), 128, kSmem, s>>>(p);
+  decode_split_kernel<<<dim3(p.splits, B * Hkv), 128, DecodeLayout::SMEM_BYTES, s>>>(tk, tv, p, err_word);
   decode_combine_kernel<<<B * H, 128, 0, s>>>(p);
   return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
 }

@@ -13,18 +13,19 @@
 // decode_combine_kernel merges the splits exactly through their maxima and
 // sums and writes O / (S l) and lse.
 //
-// With one query row per head there is no M dimension for the tensor cores:
-// products run on the FP32 pipes.  E4M3 x E4M3 products are exact in FP32.
-// Thread t owns key t of a tile for S = q K^T; for P^ V it owns the four
-// output columns 4 (t % 32) .. + 3 over the keys 32 (t / 32) .. + 31 of each
-// tile (one 32-bit load of V per key), and the four key quarters are summed
-// once per split.
-// K rows are stored with their 16-byte chunks XOR-swizzled by (row & 7), so
-// that a warp reading one chunk of 32 different rows hits 32 distinct banks.
+// The products run as tcgen05 FP8 MMAs with the keys (and, for P^ V, the
+// head dimension) as the M = 128 side and the query heads padded to N = 16:
+//   S^T [128 keys x 16]  = K [128 keys x d] . Q^T          (K K-major from TMA, Q K-major)
+//   O^T [d x 16]        += V^T [d x 128 keys] . P^^T       (V MN-major straight from TMA, P^ K-major)
+// Thread t holds key t's 16 logits (TMEM lane t of S^T) and, for the
+// rescale and the partials, column d = t of O^T.  The maxima and sums of
+// each query head run over the keys: warp shuffles, then the four warps
+// through shared memory.  S^T is double-buffered in tensor memory so the
+// next tile's product runs during this tile's softmax and P^ V.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
-#include <cuda_fp16.h>
 #include <cstdint>
 
 #include "sm100_ptx.cuh"
@@ -48,217 +49,240 @@ struct DecodeParams {
   float log2_p_scale;  // log2(S)
 };
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
+constexpr int kTcN = 16;  // query heads padded to the MMA's N
 
-// Four E4M3 bytes of a 32-bit word to float32 (exact).
-__device__ __forceinline__ void e4m3x4_to_f32(uint32_t w, float& a, float& b, float& c, float& d) {
-  uint32_t lo, hi;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(lo) : "h"(static_cast<uint16_t>(w & 0xFFFFu)));
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(hi) : "h"(static_cast<uint16_t>(w >> 16)));
-  const __half2 l2 = *reinterpret_cast<const __half2*>(&lo);
-  const __half2 h2 = *reinterpret_cast<const __half2*>(&hi);
-  a = __low2float(l2), b = __high2float(l2), c = __low2float(h2), d = __high2float(h2);
-}
+struct DecodeLayout {
+  static constexpr int OFF_K = 0;                       // 2 stages x 16 KB (TMA, 128-byte swizzle)
+  static constexpr int OFF_V = 2 * 16384;               // 2 stages x 16 KB
+  static constexpr int OFF_Q = 4 * 16384;               // Q: 16 rows x 128 B, K-major (B of S^T)
+  static constexpr int OFF_P = OFF_Q + 2048;            // P^: 16 rows x 128 keys, K-major (B of O^T)
+  static constexpr int OFF_RED = OFF_P + 2048;          // float [2][4 warps][16]: maxima, sums
+  static constexpr int OFF_BAR = OFF_RED + 2 * 4 * kTcN * 4;
+  static constexpr int SMEM_BYTES = OFF_BAR + 128 + 1024;
+};
+static_assert(DecodeLayout::OFF_Q % 1024 == 0 && DecodeLayout::OFF_P % 1024 == 0, "swizzled tiles 1024-aligned");
 
-// The E4M3 value nearest to x (round to nearest even, saturating), as float32.
-__device__ __forceinline__ float e4m3_round(float x) {
-  const uint32_t c = cvt_e4m3x2(x, 0.0f);
-  float a, b, cc, dd;
-  e4m3x4_to_f32(c, a, b, cc, dd);
-  return a;
-}
+__global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
+                                                         const __grid_constant__ CUtensorMap tm_v,
+                                                         const DecodeParams p, uint32_t* err_word) {
+  using L = DecodeLayout;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* sMax = reinterpret_cast<float*>(base + L::OFF_RED);  // [4][16]
+  float* sSum = sMax + 4 * kTcN;                               // [4][16]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
+  uint64_t* bar_kv = bars + 0;  // two stages: K and V of a tile landed
+  uint64_t* bar_s = bars + 2;   // S^T of the next tile computed
+  uint64_t* bar_o = bars + 3;   // O^T += P^ V of this tile complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
 
-__global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p) {
-  constexpr int kTile = 128 * 128;  // bytes of one K or V tile
-  extern __shared__ __align__(16) uint8_t dsm[];
-  uint8_t* sK = dsm;                            // 2 x 16 KB, swizzled rows
-  uint8_t* sV = dsm + 2 * kTile;                // 2 x 16 KB
-  float* sQ = reinterpret_cast<float*>(dsm + 4 * kTile);  // [G][128]
-  float* sP = sQ + kDecodeMaxG * 128;                     // [128 keys][8] P^ values
-  float* sRed = sP + kDecodeMaxG * 128;                   // [4 warps][G]
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int split = blockIdx.x, zkv = blockIdx.y;  // zkv = b * Hkv + hkv
   const int b = zkv / p.Hkv, hkv = zkv - b * p.Hkv;
   const int G = p.G;
   const int tile0 = split * p.split_tiles;
   const int nt = min(p.split_tiles, p.ntiles - tile0);
-  const uint8_t* kbase = p.k + static_cast<int64_t>(zkv) * p.N * 128;
-  const uint8_t* vbase = p.v + static_cast<int64_t>(zkv) * p.N * 128;
-
-  // Query rows of the G heads, decoded.
-  for (int i = t; i < G * 128; i += 128) {
-    const int g = i >> 7, c = i & 127;
-    const uint8_t code = p.q[(static_cast<int64_t>(b) * p.H + hkv * G + g) * 128 + c];
-    float a, bb, cc, dd;
-    e4m3x4_to_f32(code, a, bb, cc, dd);
-    sQ[i] = a;
-  }
-
   auto tile_of = [&](int i) { return tile0 + (p.reverse ? nt - 1 - i : i); };
-  // Issues the copies of tile `tile` into buffer `buf`; rows at or past N are zero-filled.
-  auto fetch = [&](int tile, int buf) {
-    const uint32_t dK = smem_u32(sK + buf * kTile), dV = smem_u32(sV + buf * kTile);
+
+  if (t == 0) {
+    for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 64);
+    tmem_relinquish();
+  }
+  // Q rows of the G heads (rows G..15 zero) and an all-zero P^ tile, both in
+  // the 128-byte-swizzled K-major layout: row r, 16-byte chunk c at
+  // r * 128 + ((c ^ (r & 7)) << 4).
+  {
+    const int r = t >> 3, c = t & 7;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (r < G) {
+      const uint8_t* src = p.q + (static_cast<int64_t>(b) * p.H + hkv * G + r) * 128 + c * 16;
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int i = t + 128 * r, row = i >> 3, chunk = i & 7;
-      const int key = tile * 128 + row;
-      const bool in = key < p.N;
-      const int64_t off = static_cast<int64_t>(in ? key : 0) * 128 + chunk * 16;
-      cp_async16(dK + row * 128 + ((chunk ^ (row & 7)) << 4), kbase + off, in ? 16u : 0u);
-      cp_async16(dV + row * 128 + (chunk << 4), vbase + off, in ? 16u : 0u);
+      for (int i = 0; i < 16; ++i) w[i >> 2] |= static_cast<uint32_t>(src[i]) << (8 * (i & 3));
     }
-    cp_async_commit();
+    const uint32_t off = r * 128 + ((c ^ (r & 7)) << 4);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(base + L::OFF_Q) + off), "r"(w[0]),
+                 "r"(w[1]), "r"(w[2]), "r"(w[3])
+                 : "memory");
+    asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(smem_u32(base + L::OFF_P) + off), "r"(0u)
+                 : "memory");
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t tO = tmem + 32;  // O^T: columns 32 .. 47; S^T buffers at 0 .. 15 and 16 .. 31
+
+  auto issue_tile = [&](int i) {  // K and V of the split's i-th tile into stage i % 2
+    const int st = i & 1;
+    mbar_arrive_expect_tx(bar_kv + st, 2 * 16384);
+    tma_load_3d(base + L::OFF_K + st * 16384, &tm_k, bar_kv + st, 0, tile_of(i) * 128, zkv);
+    tma_load_3d(base + L::OFF_V + st * 16384, &tm_v, bar_kv + st, 0, tile_of(i) * 128, zkv);
+  };
+  constexpr uint32_t idesc_s = idesc_e4m3_f32(128, kTcN, false, false);
+  constexpr uint32_t idesc_o = idesc_e4m3_f32(128, kTcN, true, false);  // A = V^T read MN-major
+  const uint64_t dQ = smem_desc(smem_u32(base + L::OFF_Q), 16, 1024, 2);
+  const uint64_t dP = smem_desc(smem_u32(base + L::OFF_P), 16, 1024, 2);
+  auto issue_s = [&](int i) {  // S^T of tile i into buffer i % 2 (its K must have landed)
+    const uint64_t dK = smem_desc(smem_u32(base + L::OFF_K + (i & 1) * 16384), 16, 1024, 2);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tmem + (i & 1) * 16, dK + 2 * kk, dQ + 2 * kk, idesc_s, kk > 0);
+    mma_commit(bar_s);
   };
 
-  float m[kDecodeMaxG], l[kDecodeMaxG], acc[kDecodeMaxG][4];
-#pragma unroll
-  for (int g = 0; g < kDecodeMaxG; ++g) {
-    m[g] = -INFINITY, l[g] = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[g][j] = 0.0f;
-  }
-  const float c = p.scale_log2;
-
-  fetch(tile_of(0), 0);
-  for (int i = 0; i < nt; ++i) {
-    const int buf = i & 1;
-    const int tile = tile_of(i);
-    if (i + 1 < nt) {
-      fetch(tile_of(i + 1), buf ^ 1);
-      cp_async_wait<1>();
+  bool fail = false;
+  if (t == 0) {
+    issue_tile(0);
+    if (nt > 1) issue_tile(1);
+    if (mbar_wait_bounded(bar_kv, 0, err_word, kErrTimeoutKV)) {
+      tc_fence_after();
+      issue_s(0);
     } else {
-      cp_async_wait<0>();
+      fail = true;
     }
-    __syncthreads();
-    // S for key t of this tile, against every query row.
-    float s[kDecodeMaxG];
+  }
+
+  float m[kTcN], l[kTcN];
 #pragma unroll
-    for (int g = 0; g < kDecodeMaxG; ++g) s[g] = 0.0f;
-    const uint8_t* krow = sK + buf * kTile + t * 128;
+  for (int g = 0; g < kTcN; ++g) m[g] = -INFINITY, l[g] = 0.0f;
+  const float c = p.scale_log2;
+  bool abort = false;
+
+  for (int i = 0; i < nt; ++i) {
+    const int key = tile_of(i) * 128 + t;
+    const bool valid = key < p.N;
+    // This tile's logits.
+    if (!mbar_wait_bounded(bar_s, i & 1, err_word, kErrTimeoutMMA)) fail = true;
+    tc_fence_after();
+    uint32_t rs[16];
+    tmem_ld16(tmem + (i & 1) * 16 + lane_off, rs);
+    tmem_wait_ld();
+    float s[kTcN];
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
-      const uint4 w = *reinterpret_cast<const uint4*>(krow + ((ch ^ (t & 7)) << 4));
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    for (int g = 0; g < kTcN; ++g) s[g] = __uint_as_float(rs[g]);
+    // Tile maximum of every query head: warp, then the four warps.
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float k0, k1, k2, k3;
-        e4m3x4_to_f32(ws[j], k0, k1, k2, k3);
-        const int col = ch * 16 + j * 4;
-#pragma unroll
-        for (int g = 0; g < kDecodeMaxG; ++g) {
-          if (g < G) {
-            const float* qg = sQ + g * 128 + col;
-            s[g] = fmaf(k0, qg[0], s[g]);
-            s[g] = fmaf(k1, qg[1], s[g]);
-            s[g] = fmaf(k2, qg[2], s[g]);
-            s[g] = fmaf(k3, qg[3], s[g]);
-          }
-        }
-      }
-    }
-    const bool valid = tile * 128 + t < p.N;
-    // Tile maximum of every row: warp, then across the four warps.
-#pragma unroll
-    for (int g = 0; g < kDecodeMaxG; ++g) {
+    for (int g = 0; g < kTcN; ++g) {
       if (g < G) {
         float x = valid ? s[g] : -INFINITY;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-        if (lane == 0) sRed[warp * kDecodeMaxG + g] = x;
+        if (lane == 0) sMax[warp * kTcN + g] = x;
       }
     }
-    __syncthreads();
-    float alpha[kDecodeMaxG];
+    // The previous P^ V must be complete before P^ and O^T are touched; its
+    // stage is then free for the tile after next.
+    if (i > 0) {
+      if (!mbar_wait_bounded(bar_o, (i - 1) & 1, err_word, kErrTimeoutMMA)) fail = true;
+      tc_fence_after();
+      if (t == 0 && !fail && i + 1 < nt) issue_tile(i + 1);
+    }
+    abort = __syncthreads_or(fail) != 0;
+    if (abort) break;
+    float alpha[kTcN];
+    bool any_rescale = false;
 #pragma unroll
-    for (int g = 0; g < kDecodeMaxG; ++g) {
+    for (int g = 0; g < kTcN; ++g) {
       alpha[g] = 1.0f;
       if (g < G) {
-        const float tmax = fmaxf(fmaxf(sRed[g], sRed[kDecodeMaxG + g]),
-                                 fmaxf(sRed[2 * kDecodeMaxG + g], sRed[3 * kDecodeMaxG + g]));
+        const float tmax = fmaxf(fmaxf(sMax[g], sMax[kTcN + g]), fmaxf(sMax[2 * kTcN + g], sMax[3 * kTcN + g]));
         const float m_new = fmaxf(m[g], tmax * c);
         alpha[g] = (m_new == m[g]) ? 1.0f : ex2_approx(m[g] - m_new);
+        any_rescale |= alpha[g] != 1.0f;
         m[g] = m_new;
         // P * S for key t: the scale enters the exponent; masked keys give 0.
         const float ps = valid ? ex2_approx(fmaf(s[g], c, p.log2_p_scale - m_new)) : 0.0f;
         s[g] = ps;
-        sP[t * kDecodeMaxG + g] = e4m3_round(ps);
+        const uint32_t code = cvt_e4m3x2(ps, 0.0f) & 0xFFu;
+        const uint32_t off = g * 128 + ((((t >> 4) ^ (g & 7))) << 4) + (t & 15);
+        asm volatile("st.shared.u8 [%0], %1;" ::"r"(smem_u32(base + L::OFF_P) + off), "r"(code) : "memory");
       }
     }
-    __syncthreads();  // every thread has read sRed (maxima) and written sP
+    // Row sums of the unquantised P * S.
 #pragma unroll
-    for (int g = 0; g < kDecodeMaxG; ++g) {
+    for (int g = 0; g < kTcN; ++g) {
       if (g < G) {
         float x = s[g];
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-        if (lane == 0) sRed[warp * kDecodeMaxG + g] = x;
+        if (lane == 0) sSum[warp * kTcN + g] = x;
       }
     }
-    // P^ V: columns 4 cg .. 4 cg + 3 over this thread's quarter of the keys.
+    // O^T *= alpha per query head (column), when any maximum grew; every
+    // thread computed the same alphas.
+    if (i > 0 && any_rescale) {
+      uint32_t o[16];
+      tmem_ld16(tO + lane_off, o);
+      tmem_wait_ld();
 #pragma unroll
-    for (int g = 0; g < kDecodeMaxG; ++g) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[g][j] *= alpha[g];
+      for (int g = 0; g < kTcN; ++g) o[g] = __float_as_uint(__uint_as_float(o[g]) * alpha[g]);
+      tmem_st16(tO + lane_off, o);
+      tmem_wait_st();
     }
-    const uint8_t* vtile = sV + buf * kTile + (lane << 2);
-#pragma unroll 4
-    for (int kk = 0; kk < 32; ++kk) {
-      const int key = (warp << 5) + kk;
-      float v0, v1, v2, v3;
-      e4m3x4_to_f32(*reinterpret_cast<const uint32_t*>(vtile + key * 128), v0, v1, v2, v3);
-      const float4 pa = *reinterpret_cast<const float4*>(sP + key * kDecodeMaxG);
-      const float4 pb = *reinterpret_cast<const float4*>(sP + key * kDecodeMaxG + 4);
-      const float pg[kDecodeMaxG] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
 #pragma unroll
-      for (int g = 0; g < kDecodeMaxG; ++g) {
-        if (g < G) {
-          acc[g][0] = fmaf(pg[g], v0, acc[g][0]);
-          acc[g][1] = fmaf(pg[g], v1, acc[g][1]);
-          acc[g][2] = fmaf(pg[g], v2, acc[g][2]);
-          acc[g][3] = fmaf(pg[g], v3, acc[g][3]);
-        }
-      }
-    }
-    __syncthreads();  // sums in sRed; every read of sP and of this buffer done
-#pragma unroll
-    for (int g = 0; g < kDecodeMaxG; ++g) {
+    for (int g = 0; g < kTcN; ++g) {
       if (g < G) {
-        const float tsum = (sRed[g] + sRed[kDecodeMaxG + g]) + (sRed[2 * kDecodeMaxG + g] + sRed[3 * kDecodeMaxG + g]);
+        const float tsum = (sSum[g] + sSum[kTcN + g]) + (sSum[2 * kTcN + g] + sSum[3 * kTcN + g]);
         l[g] = l[g] * alpha[g] + tsum;  // l * S
       }
     }
-    __syncthreads();  // sRed is rewritten by the next tile's maxima
-  }
-  // Sum of the four key quarters (through the K buffers, free now), then
-  // the partial results of this split.
-  float* sAcc = reinterpret_cast<float*>(dsm);  // [4 quarters][G][128]
+    if (t == 0) {
+      tc_fence_after();
+      // O^T += V^T P^^T: V stage i % 2 read MN-major (32 keys = 32 rows of 128 B per step).
+      const uint64_t dV = smem_desc(smem_u32(base + L::OFF_V + (i & 1) * 16384), 16384, 1024, 2);
 #pragma unroll
-  for (int g = 0; g < kDecodeMaxG; ++g) {
-    if (g < G) {
-      *reinterpret_cast<float4*>(sAcc + (warp * kDecodeMaxG + g) * 128 + (lane << 2)) =
-          make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
-    }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int g = 0; g < kDecodeMaxG; ++g) {
-    if (g < G) {
-      const float sum = (sAcc[(0 * kDecodeMaxG + g) * 128 + t] + sAcc[(1 * kDecodeMaxG + g) * 128 + t]) +
-                        (sAcc[(2 * kDecodeMaxG + g) * 128 + t] + sAcc[(3 * kDecodeMaxG + g) * 128 + t]);
-      float* dst = p.part + (static_cast<int64_t>(b * p.H + hkv * G + g) * p.splits + split) * kDecodePartStride;
-      dst[t] = sum;
-      if (t == 0) {
-        dst[128] = m[g];
-        dst[129] = l[g];
+      for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tO, dV + 256 * kk, dP + 2 * kk, idesc_o, (i > 0) || (kk > 0));
+      mma_commit(bar_o);
+      if (i + 1 < nt) {
+        if (mbar_wait_bounded(bar_kv + ((i + 1) & 1), ((i + 1) >> 1) & 1, err_word, kErrTimeoutKV)) {
+          tc_fence_after();
+          issue_s(i + 1);
+        } else {
+          fail = true;
+        }
       }
     }
+    // The sums are read before the next tile rewrites them: the next
+    // tile's first barrier comes after its maxima, and the sums after it.
+  }
+  abort = __syncthreads_or(fail || abort) != 0;
+  if (!abort && nt > 0) {
+    if (!mbar_wait_bounded(bar_o, (nt - 1) & 1, err_word, kErrTimeoutMMA)) abort = true;
+    tc_fence_after();
+  }
+  abort = __syncthreads_or(abort) != 0;
+  if (!abort) {
+    // Partials of this split: column d = t of O^T for every query head.
+    uint32_t o[16];
+    tmem_ld16(tO + lane_off, o);
+    tmem_wait_ld();
+#pragma unroll
+    for (int g = 0; g < kTcN; ++g) {
+      if (g < G) {
+        float* dst = p.part + (static_cast<int64_t>(b * p.H + hkv * G + g) * p.splits + split) * kDecodePartStride;
+        dst[t] = __uint_as_float(o[g]);
+        if (t == 0) {
+          dst[128] = m[g];
+          dst[129] = l[g];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
   }
 }
 

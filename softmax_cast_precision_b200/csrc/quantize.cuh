@@ -80,9 +80,11 @@ __device__ __forceinline__ uint32_t quant_word(const uint4& q, int i) {
 }
 
 // The thread's E values of the row as float32, with the signs and the
-// rotation applied when enabled.
+// unnormalised transform x H_d applied when the rotation is enabled (the
+// factor 1/sqrt(d) is applied by the caller).  `sb` holds this thread's E
+// sign bits (bit e set: element e is negated).
 template <int E>
-__device__ __forceinline__ void quant_transform_row(const QuantParams& p, const RowBits<E>& r, int part,
+__device__ __forceinline__ void quant_transform_row(const QuantParams& p, const RowBits<E>& r, int part, uint32_t sb,
                                                     float (&v)[E]) {
   if (p.x_f32) {
 #pragma unroll
@@ -97,54 +99,63 @@ __device__ __forceinline__ void quant_transform_row(const QuantParams& p, const 
     }
   }
   if (!p.rotate) return;
-  // This thread's E sign bits: E = 32 is one whole word, E = 16 half of one.
-  const int i0 = part * E;
-  const int wi = i0 >> 5;
-  const uint32_t sb = (wi == 0 ? p.sign_bits[0] : wi == 1 ? p.sign_bits[1] : wi == 2 ? p.sign_bits[2] : p.sign_bits[3]) >>
-                      (i0 & 31);
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     if ((sb >> e) & 1u) v[e] = -v[e];
   }
-  // Stages inside the thread.
+  // Stage h = 1 inside the thread, one rounding per sum or difference.
 #pragma unroll
-  for (int h = 1; h < E; h *= 2) {
+  for (int e = 0; e < E; e += 2) {
+    const float a = v[e], b = v[e + 1];
+    v[e] = a + b;
+    v[e + 1] = a - b;
+  }
+  // Stages h = 2 .. E/2: both members of a pair (e, e + 1) meet (e + h, e + 1 + h), in packed f32x2.
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
+  for (int h = 2; h < E; h *= 2) {
+#pragma unroll
+    for (int e = 0; e < E; e += 2) {
       if ((e & h) == 0) {
-        const float a = v[e], b = v[e + h];
-        v[e] = a + b;
-        v[e + h] = a - b;
+        const uint64_t a = f2_pack(v[e], v[e + 1]), b = f2_pack(v[e + h], v[e + 1 + h]);
+        f2_unpack(f2_add(a, b), v[e], v[e + 1]);
+        f2_unpack(f2_add(a, f2_mul(b, f2_pack(-1.0f, -1.0f))), v[e + h], v[e + 1 + h]);
       }
     }
   }
   // The two stages across the row's four threads: the partner of element
-  // i = part*E + e is i ^ h, in part ^ (h / E) at the same e.
+  // i = part*E + e is i ^ h, in part ^ (h / E) at the same e; the lower
+  // member keeps v + other, the upper other - v (one rounding each).
 #pragma unroll
   for (int hp = 1; hp < kQuantThreadsPerRow; hp *= 2) {
-    const bool upper = (part & hp) != 0;
+    const float sg = (part & hp) ? -1.0f : 1.0f;
+    const uint64_t sg2 = f2_pack(sg, sg);
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const float other = __shfl_xor_sync(0xffffffffu, v[e], hp);
-      v[e] = upper ? (other - v[e]) : (v[e] + other);
+    for (int e = 0; e < E; e += 2) {
+      const float o0 = __shfl_xor_sync(0xffffffffu, v[e], hp);
+      const float o1 = __shfl_xor_sync(0xffffffffu, v[e + 1], hp);
+      f2_unpack(f2_fma(f2_pack(v[e], v[e + 1]), sg2, f2_pack(o0, o1)), v[e], v[e + 1]);
     }
   }
-  const float inv_sqrt_d = (E == 32) ? 0.08838834764831845f : 0.125f;  // float32(1/sqrt(d)), d = 128 or 64
-#pragma unroll
-  for (int e = 0; e < E; ++e) v[e] *= inv_sqrt_d;
 }
 
+// Stores E4M3(v * mul): mul = c / s, with c = float32(1/sqrt(d)) after a
+// rotation (else 1) and s the block's power-of-two descale, so that
+// v * mul = (v * c) / s exactly (s is a power of two).
 template <int E>
 __device__ __forceinline__ void quant_store_row(const QuantParams& p, int z, int row, int part, const float (&v)[E],
-                                                float inv_s) {
+                                                float mul) {
   uint4* dst = reinterpret_cast<uint4*>(p.xq + (static_cast<int64_t>(z) * p.N + row) * p.d + part * E);
+  const uint64_t m2 = f2_pack(mul, mul);
 #pragma unroll
   for (int c = 0; c < E / 16; ++c) {
     uint32_t w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int e = c * 16 + 4 * j;
-      w[j] = cvt_e4m3x2(v[e] * inv_s, v[e + 1] * inv_s) | (cvt_e4m3x2(v[e + 2] * inv_s, v[e + 3] * inv_s) << 16);
+      float a, b, cc, dd;
+      f2_unpack(f2_mul(f2_pack(v[e], v[e + 1]), m2), a, b);
+      f2_unpack(f2_mul(f2_pack(v[e + 2], v[e + 3]), m2), cc, dd);
+      w[j] = cvt_e4m3x4(a, b, cc, dd);
     }
     dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
   }
@@ -156,7 +167,7 @@ __device__ __forceinline__ void quant_store_row(const QuantParams& p, int z, int
 //         p.scales[z] (float bits of a value >= 0 order like integers).
 // MODE 2: per-slab pass 2 -- cast with the descale of the slab's amax.
 template <int E, int MODE>
-__global__ void __launch_bounds__(kQuantWarps * 32) quantize_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const QuantParams p) {
   constexpr int kPasses = 128 / kQuantRowsPerPass;  // rows per thread held in registers (block_rows <= 128)
   __shared__ float warp_amax[kQuantWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -178,6 +189,18 @@ __global__ void __launch_bounds__(kQuantWarps * 32) quantize_kernel(const QuantP
       for (int j = 0; j < E / 4; ++j) raw[i].w[j] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
+  // This thread's E sign bits: E = 32 is one whole word, E = 16 half of one.
+  uint32_t sb;
+  {
+    const int i0 = part * E;
+    const int wi = i0 >> 5;
+    sb = (wi == 0 ? p.sign_bits[0] : wi == 1 ? p.sign_bits[1] : wi == 2 ? p.sign_bits[2] : p.sign_bits[3]) >>
+         (i0 & 31);
+  }
+  // float32(1/sqrt(d)) after a rotation: applied to the block maximum here
+  // (positive scaling is monotone, so max |v c| = max|v| c) and folded into
+  // the cast's multiplier.
+  const float cnorm = p.rotate ? ((E == 32) ? 0.08838834764831845f : 0.125f) : 1.0f;
   float v[kPasses][E];
   float amax = 0.0f;
 #pragma unroll
@@ -185,12 +208,13 @@ __global__ void __launch_bounds__(kQuantWarps * 32) quantize_kernel(const QuantP
     // Every lane transforms (rows past the block's end hold zeros), so the
     // full-warp shuffles of the rotation always have all 32 lanes.
     const int r = rsub + i * kQuantRowsPerPass;
-    quant_transform_row<E>(p, raw[i], part, v[i]);
+    quant_transform_row<E>(p, raw[i], part, sb, v[i]);
     if (r < rows) {
 #pragma unroll
       for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(v[i][e]));
     }
   }
+  amax *= cnorm;
   int e;
   if constexpr (MODE == 2) {
     e = quant_scale_exponent(__uint_as_float(reinterpret_cast<const uint32_t*>(p.scales)[z]));
@@ -209,11 +233,11 @@ __global__ void __launch_bounds__(kQuantWarps * 32) quantize_kernel(const QuantP
     e = quant_scale_exponent(a);
     if (threadIdx.x == 0) p.scales[static_cast<int64_t>(z) * p.nblocks + blk] = ldexpf(1.0f, e);
   }
-  const float inv_s = ldexpf(1.0f, -e);  // 1 / s, exact
+  const float mul = cnorm * ldexpf(1.0f, -e);  // c / s, exact (s a power of two)
 #pragma unroll
   for (int i = 0; i < kPasses; ++i) {
     const int r = rsub + i * kQuantRowsPerPass;
-    if (r < rows) quant_store_row<E>(p, z, r0 + r, part, v[i], inv_s);
+    if (r < rows) quant_store_row<E>(p, z, r0 + r, part, v[i], mul);
   }
 }
 
