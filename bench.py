@@ -82,6 +82,9 @@ def parse_args():
                          "split one problem's kv heads and all-gather the output (strong scaling)")
     ap.add_argument("--skip-cpu-baseline", action="store_true",
                     help="omit the oracle timing (used under ncu)")
+    ap.add_argument("--head-dim", type=int, default=None, choices=[64, 128],
+                    help="run the fp8 path's prefill with this head dimension (64: the 64-key-block kernel; a "
+                         "profiling case, not the headline)")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="run the fp8 path's prefill at this sequence length instead of 32768 (a smaller case "
                          "for profiling; not the headline workload)")
@@ -971,6 +974,15 @@ def set_seq_len(args):
     BWD_WORKLOAD_DESC = BWD_WORKLOAD_DESC.replace("N=32768", tag)
 
 
+def set_head_dim(args):
+    """The fp8 path's prefill at another head dimension (--head-dim; profiling)."""
+    global WORKLOAD, WORKLOAD_DESC
+    if args.impl != "ours" or args.shard != "replicas" or args.path != "fp8":
+        raise SystemExit("--head-dim covers our fp8 path with replicas")
+    WORKLOAD = dataclasses.replace(WORKLOAD, d=args.head_dim)
+    WORKLOAD_DESC = WORKLOAD_DESC.replace("d=128", f"d={args.head_dim} (profiling case, not the headline)")
+
+
 def main():
     args = parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -980,6 +992,8 @@ def main():
         raise SystemExit("--warmup must be >= 3")
     if args.seq_len is not None:
         set_seq_len(args)
+    if args.head_dim is not None:
+        set_head_dim(args)
     if args.impl == "reference":
         if args.path in ("bf16qk", "decode", "bwd"):
             raise SystemExit("--impl reference covers --path fp8 and wide")

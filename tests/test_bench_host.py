@@ -89,6 +89,7 @@ def test_peak_falls_back_without_the_measured_file(tmp_path, monkeypatch):
     (["--warmup", "2"], "--warmup must be >= 3"),
     (["--seq-len", "4096", "--impl", "reference"], "--seq-len covers"),
     (["--seq-len", "4096", "--shard", "heads"], "--seq-len covers"),
+    (["--head-dim", "64", "--path", "bwd"], "--head-dim covers"),
 ])
 def test_dispatch_guards_exit_before_any_device_work(argv, message, monkeypatch):
     monkeypatch.setattr("sys.argv", ["bench.py", *argv])
