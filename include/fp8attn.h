@@ -115,8 +115,11 @@ int fp8attn_pzero_count(const void* q, const void* k, const void* v,
  * with max|x| <= 448 s, so that x = s * E4M3 code up to the cast's rounding
  * and nothing saturates.  Blocks are block_rows (1..128) consecutive rows of
  * one slab, scales is then a device float array [Z, ceil(N / block_rows)];
- * block_rows = 0 gives one descale per slab, scales [Z] (three launches; the
- * array holds intermediate maxima until the last one).  d must be 64 or 128.
+ * block_rows = 0 gives one descale per slab, scales [Z]: an amax pass, a
+ * cast pass, and one launch that turns the maxima into descales (the array
+ * holds intermediate maxima until that last launch).
+ * d must be 64 or 128, and Z * ceil(N / block_rows) at most 2^30
+ * (FP8ATTN_ERR_UNSUPPORTED otherwise).
  * For fp8attn_fwd_scaled: Q and K with block_rows = 128, V with 0, the same
  * signs for all three.
  */

@@ -12,6 +12,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 
@@ -419,23 +420,34 @@ extern "C" int fp8attn_fwd_noalloc(const void* q, const void* k, const void* v, 
 namespace fp8attn {
 namespace {
 
+template <int E, int MODE>
+int launch_quantize_ring(const QuantParams& p, cudaStream_t s, uint32_t* err_word) {
+  const int nunits = p.Z * p.nblocks;
+  if (nunits == 0) return FP8ATTN_OK;
+  const int smem = quant_stages(p) * quant_stage_bytes(p);
+  if (cudaFuncSetAttribute(quantize_kernel<E, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return FP8ATTN_ERR_CUDA;
+  const int sms = num_sms();
+  if (sms <= 0) return FP8ATTN_ERR_CUDA;
+  const int grid = std::min(nunits, 2 * sms);
+  quantize_kernel<E, MODE><<<grid, kQuantWarps * 32, smem, s>>>(p, err_word);
+  return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
+}
+
 template <int E>
 int launch_quantize(QuantParams p, cudaStream_t s) {
-  const dim3 block(kQuantWarps * 32);
-  if (p.block_rows > 0) {
-    const dim3 grid((p.N + p.block_rows - 1) / p.block_rows, p.Z);
-    if (grid.x > 0) quantize_kernel<E, 0><<<grid, block, 0, s>>>(p);
-  } else {
-    if (cudaMemsetAsync(p.scales, 0, sizeof(float) * static_cast<size_t>(p.Z), s) != cudaSuccess)
-      return FP8ATTN_ERR_CUDA;
-    p.block_rows = 128;
-    const dim3 grid((p.N + 127) / 128, p.Z);
-    if (grid.x > 0) {
-      quantize_kernel<E, 1><<<grid, block, 0, s>>>(p);
-      quantize_kernel<E, 2><<<grid, block, 0, s>>>(p);
-    }
-    quantize_finish_kernel<<<(p.Z + 255) / 256, 256, 0, s>>>(p.scales, p.Z);
-  }
+  uint32_t* err_word = nullptr;
+  if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err_word), g_error_word) != cudaSuccess) return FP8ATTN_ERR_CUDA;
+  if (p.block_rows > 0) return launch_quantize_ring<E, 0>(p, s, err_word);
+  if (cudaMemsetAsync(p.scales, 0, sizeof(float) * static_cast<size_t>(p.Z), s) != cudaSuccess)
+    return FP8ATTN_ERR_CUDA;
+  p.block_rows = 128;
+  p.nblocks = (p.N + 127) / 128;
+  int st = launch_quantize_ring<E, 1>(p, s, err_word);
+  if (st == FP8ATTN_OK) st = launch_quantize_ring<E, 2>(p, s, err_word);
+  if (st != FP8ATTN_OK) return st;
+  quantize_finish_kernel<<<(p.Z + 255) / 256, 256, 0, s>>>(p.scales, p.Z);
   return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
 }
 
@@ -466,6 +478,8 @@ extern "C" int fp8attn_quantize(const void* x, int x_dtype, void* xq, float* sca
   p.d = d;
   p.block_rows = block_rows;
   p.nblocks = block_rows > 0 ? (N + block_rows - 1) / block_rows : 1;
+  // The persistent CTAs number the blocks of all slabs in 32-bit integers.
+  if (block_rows > 0 && static_cast<int64_t>(Z) * p.nblocks > (int64_t(1) << 30)) return FP8ATTN_ERR_UNSUPPORTED;
   p.x_f32 = x_dtype;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d == 128 ? launch_quantize<32>(p, s) : launch_quantize<16>(p, s);

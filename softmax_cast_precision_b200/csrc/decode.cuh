@@ -49,12 +49,13 @@ struct DecodeParams {
   float log2_p_scale;  // log2(S)
 };
 
-constexpr int kTcN = 16;  // query heads padded to the MMA's N
+constexpr int kTcN = 16;         // query heads padded to the MMA's N
+constexpr int kDecodeStages = 2;  // K/V ring: tile i + 1 loads while tile i is consumed
 
 struct DecodeLayout {
-  static constexpr int OFF_K = 0;                       // 2 stages x 16 KB (TMA, 128-byte swizzle)
-  static constexpr int OFF_V = 2 * 16384;               // 2 stages x 16 KB
-  static constexpr int OFF_Q = 4 * 16384;               // Q: 16 rows x 128 B, K-major (B of S^T)
+  static constexpr int OFF_K = 0;                                 // kDecodeStages x 16 KB (TMA, 128-byte swizzle)
+  static constexpr int OFF_V = kDecodeStages * 16384;             // kDecodeStages x 16 KB
+  static constexpr int OFF_Q = 2 * kDecodeStages * 16384;         // Q: 16 rows x 128 B, K-major (B of S^T)
   static constexpr int OFF_P = OFF_Q + 2048;            // P^: 16 rows x 128 keys, K-major (B of O^T)
   static constexpr int OFF_RED = OFF_P + 2048;          // float [2][4 warps][16]: maxima, sums
   static constexpr int OFF_BAR = OFF_RED + 2 * 4 * kTcN * 4;
@@ -71,10 +72,11 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
   float* sMax = reinterpret_cast<float*>(base + L::OFF_RED);  // [4][16]
   float* sSum = sMax + 4 * kTcN;                               // [4][16]
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
-  uint64_t* bar_kv = bars + 0;  // two stages: K and V of a tile landed
-  uint64_t* bar_s = bars + 2;   // S^T of the next tile computed
-  uint64_t* bar_o = bars + 3;   // O^T += P^ V of this tile complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  uint64_t* bar_kv = bars + 0;               // per stage: K and V of a tile landed
+  uint64_t* bar_s = bars + kDecodeStages;     // S^T of the next tile computed
+  uint64_t* bar_o = bars + kDecodeStages + 1; // O^T += P^ V of this tile complete
+  uint64_t* bar_drain = bars + kDecodeStages + 2;  // every product issued so far complete (abort path)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kDecodeStages + 3);
 
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int split = blockIdx.x, zkv = blockIdx.y;  // zkv = b * Hkv + hkv
@@ -85,7 +87,7 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
   auto tile_of = [&](int i) { return tile0 + (p.reverse ? nt - 1 - i : i); };
 
   if (t == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < kDecodeStages + 3; ++i) mbar_init(bars + i, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -120,8 +122,10 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
   const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t tO = tmem + 32;  // O^T: columns 32 .. 47; S^T buffers at 0 .. 15 and 16 .. 31
 
-  auto issue_tile = [&](int i) {  // K and V of the split's i-th tile into stage i % 2
-    const int st = i & 1;
+  int issued = 0, landed = 0;     // thread 0: tiles whose loads were issued / waited for
+  auto issue_tile = [&](int i) {  // K and V of the split's i-th tile into stage i % kDecodeStages
+    const int st = i % kDecodeStages;
+    issued = i + 1;
     mbar_arrive_expect_tx(bar_kv + st, 2 * 16384);
     tma_load_3d(base + L::OFF_K + st * 16384, &tm_k, bar_kv + st, 0, tile_of(i) * 128, zkv);
     tma_load_3d(base + L::OFF_V + st * 16384, &tm_v, bar_kv + st, 0, tile_of(i) * 128, zkv);
@@ -130,8 +134,8 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
   constexpr uint32_t idesc_o = idesc_e4m3_f32(128, kTcN, true, false);  // A = V^T read MN-major
   const uint64_t dQ = smem_desc(smem_u32(base + L::OFF_Q), 16, 1024, 2);
   const uint64_t dP = smem_desc(smem_u32(base + L::OFF_P), 16, 1024, 2);
-  auto issue_s = [&](int i) {  // S^T of tile i into buffer i % 2 (its K must have landed)
-    const uint64_t dK = smem_desc(smem_u32(base + L::OFF_K + (i & 1) * 16384), 16, 1024, 2);
+  auto issue_s = [&](int i) {  // S^T of tile i into TMEM buffer i % 2 (its K must have landed)
+    const uint64_t dK = smem_desc(smem_u32(base + L::OFF_K + (i % kDecodeStages) * 16384), 16, 1024, 2);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tmem + (i & 1) * 16, dK + 2 * kk, dQ + 2 * kk, idesc_s, kk > 0);
     mma_commit(bar_s);
@@ -139,9 +143,9 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
 
   bool fail = false;
   if (t == 0) {
-    issue_tile(0);
-    if (nt > 1) issue_tile(1);
+    for (int i = 0; i < kDecodeStages && i < nt; ++i) issue_tile(i);
     if (mbar_wait_bounded(bar_kv, 0, err_word, kErrTimeoutKV)) {
+      landed = 1;
       tc_fence_after();
       issue_s(0);
     } else {
@@ -178,11 +182,11 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
       }
     }
     // The previous P^ V must be complete before P^ and O^T are touched; its
-    // stage is then free for the tile after next.
+    // stage is then free for tile i - 1 + kDecodeStages.
     if (i > 0) {
       if (!mbar_wait_bounded(bar_o, (i - 1) & 1, err_word, kErrTimeoutMMA)) fail = true;
       tc_fence_after();
-      if (t == 0 && !fail && i + 1 < nt) issue_tile(i + 1);
+      if (t == 0 && !fail && i - 1 + kDecodeStages < nt) issue_tile(i - 1 + kDecodeStages);
     }
     abort = __syncthreads_or(fail) != 0;
     if (abort) break;
@@ -238,13 +242,15 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
     }
     if (t == 0) {
       tc_fence_after();
-      // O^T += V^T P^^T: V stage i % 2 read MN-major (32 keys = 32 rows of 128 B per step).
-      const uint64_t dV = smem_desc(smem_u32(base + L::OFF_V + (i & 1) * 16384), 16384, 1024, 2);
+      // O^T += V^T P^^T: V stage i % kDecodeStages read MN-major (32 keys = 32 rows of 128 B per step).
+      const uint64_t dV = smem_desc(smem_u32(base + L::OFF_V + (i % kDecodeStages) * 16384), 16384, 1024, 2);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tO, dV + 256 * kk, dP + 2 * kk, idesc_o, (i > 0) || (kk > 0));
       mma_commit(bar_o);
       if (i + 1 < nt) {
-        if (mbar_wait_bounded(bar_kv + ((i + 1) & 1), ((i + 1) >> 1) & 1, err_word, kErrTimeoutKV)) {
+        const int st = (i + 1) % kDecodeStages;
+        if (mbar_wait_bounded(bar_kv + st, ((i + 1) / kDecodeStages) & 1, err_word, kErrTimeoutKV)) {
+          landed = i + 2;
           tc_fence_after();
           issue_s(i + 1);
         } else {
@@ -277,6 +283,15 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
         }
       }
     }
+  }
+  if (abort && t == 0) {
+    // A wait ran out: let this CTA's products and tile loads still in flight
+    // land before its tensor and shared memory are released (each wait again
+    // bounded).
+    mma_commit(bar_drain);
+    mbar_wait_bounded(bar_drain, 0, err_word, kErrTimeoutMMA, 100000000ull);
+    for (int j = landed; j < issued; ++j)
+      mbar_wait_bounded(bar_kv + j % kDecodeStages, (j / kDecodeStages) & 1, err_word, kErrTimeoutKV, 100000000ull);
   }
   tc_fence_before();
   __syncthreads();

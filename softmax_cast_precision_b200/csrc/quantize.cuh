@@ -5,13 +5,23 @@
 // "FA3: Meccanica della tramoggia", point 3: a random rotation spreads
 // outlier channels over all coordinates before block quantisation).
 //
-// Four threads own one row: thread part t (0..3) holds elements
-// [t*E, t*E + E), E = d / 4, so a warp covers eight consecutive rows with
-// contiguous 16-byte loads and stores.  The rotation is the radix-2 fast
-// transform with stages of half-width 1, 2, ..., d/2 (pair i, i + h: sum at
-// i, difference at i + h); stages below E stay inside a thread, the last two
-// pair threads through shuffles.  Every operation rounds to float32 once, in
-// that fixed order.
+// The pass is a stream: each block's rows are contiguous in memory, so a
+// persistent CTA pulls whole blocks into a ring of shared-memory stages with
+// untiled bulk copies (one elected thread issues them, an mbarrier per stage
+// counts the bytes), and its 256 threads transform, reduce and cast one block
+// while the next ones are in flight.  A stage is handed back to the copy
+// engine at the block's amax barrier, when every thread has its rows in
+// registers.
+//
+// Four threads own one row.  The row is cut into 8-element chunks and thread
+// part t (0..3) holds chunks t, t + 4, t + 8, ... (E = d / 4 elements), so the
+// index of element i splits as i = 32 k + 8 t + j: j (bits 0-2) and k (bits
+// 5 and up) lie inside a thread, t (bits 3-4) across the row's four lanes.
+// The rotation is the radix-2 fast transform with stages of half-width 1, 2,
+// ..., d/2, in that order (pair i, i + h: sum at i, difference at i + h):
+// half-widths 1, 2, 4 inside the thread, 8 and 16 through shuffles, 32 and 64
+// inside the thread again.  Every operation rounds to float32 once, in that
+// fixed order.
 //
 // Descale of a block: the smallest power of two s >= 2^-126 with
 // amax <= 448 s; with amax = m 2^E (m in [1, 2)) that is 2^(E - 8) when
@@ -41,6 +51,8 @@ struct QuantParams {
 constexpr int kQuantWarps = 8;
 constexpr int kQuantThreadsPerRow = 4;
 constexpr int kQuantRowsPerPass = kQuantWarps * 32 / kQuantThreadsPerRow;  // 64
+constexpr int kQuantMaxStages = 8;
+constexpr int kQuantStageBudget = 96 * 1024;  // shared bytes of the ring (two CTAs per SM)
 
 // Binary exponent e of the descale s = 2^e of a block whose largest
 // magnitude is amax (e = 0 for an all-zero block).
@@ -52,79 +64,79 @@ __device__ __forceinline__ int quant_scale_exponent(float amax) {
   return e < -126 ? -126 : e;
 }
 
-// Raw 16-byte words of one thread's E elements of a row: bfloat16 E/8 words,
-// float32 E/4.
+// One thread's E elements of a row, read from the staged block: chunk c
+// (elements 8c .. 8c + 7 of the thread's list) is row element 32 c + 8 part.
+// Rows past the block's end read as zeros.
 template <int E>
-struct RowBits {
-  uint4 w[E / 4];
-};
-
-template <int E>
-__device__ __forceinline__ RowBits<E> quant_fetch_row(const QuantParams& p, int z, int row, int part) {
-  RowBits<E> r;
-  const int64_t base = (static_cast<int64_t>(z) * p.N + row) * p.d + part * E;
-  if (p.x_f32) {
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const float*>(p.x) + base);
+__device__ __forceinline__ void quant_read_row(const uint8_t* stage, int row_bytes, int r, int rows, int part,
+                                               int x_f32, float (&v)[E]) {
+  if (r >= rows) {
 #pragma unroll
-    for (int i = 0; i < E / 4; ++i) r.w[i] = __ldg(src + i);
-  } else {
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(p.x) + base);
-#pragma unroll
-    for (int i = 0; i < E / 8; ++i) r.w[i] = __ldg(src + i);
+    for (int e = 0; e < E; ++e) v[e] = 0.0f;
+    return;
   }
-  return r;
-}
-
-__device__ __forceinline__ uint32_t quant_word(const uint4& q, int i) {
-  return i == 0 ? q.x : i == 1 ? q.y : i == 2 ? q.z : q.w;
-}
-
-// The thread's E values of the row as float32, with the signs and the
-// unnormalised transform x H_d applied when the rotation is enabled (the
-// factor 1/sqrt(d) is applied by the caller).  `sb` holds this thread's E
-// sign bits (bit e set: element e is negated).
-template <int E>
-__device__ __forceinline__ void quant_transform_row(const QuantParams& p, const RowBits<E>& r, int part, uint32_t sb,
-                                                    float (&v)[E]) {
-  if (p.x_f32) {
+  if (x_f32) {
+    const float* src = reinterpret_cast<const float*>(stage + static_cast<int64_t>(r) * row_bytes) + 8 * part;
 #pragma unroll
-    for (int e = 0; e < E; ++e) v[e] = __uint_as_float(quant_word(r.w[e / 4], e % 4));
+    for (int c = 0; c < E / 8; ++c) {
+      const float4 a = *reinterpret_cast<const float4*>(src + 32 * c);
+      const float4 b = *reinterpret_cast<const float4*>(src + 32 * c + 4);
+      v[8 * c + 0] = a.x; v[8 * c + 1] = a.y; v[8 * c + 2] = a.z; v[8 * c + 3] = a.w;
+      v[8 * c + 4] = b.x; v[8 * c + 5] = b.y; v[8 * c + 6] = b.z; v[8 * c + 7] = b.w;
+    }
   } else {
     // bfloat16 -> float32 is exact: the 16 bits become the high half.
+    const uint16_t* src = reinterpret_cast<const uint16_t*>(stage + static_cast<int64_t>(r) * row_bytes) + 8 * part;
 #pragma unroll
-    for (int e = 0; e < E; e += 2) {
-      const uint32_t w = quant_word(r.w[e / 8], (e / 2) % 4);
-      v[e] = __uint_as_float(w << 16);
-      v[e + 1] = __uint_as_float(w & 0xFFFF0000u);
-    }
-  }
-  if (!p.rotate) return;
+    for (int c = 0; c < E / 8; ++c) {
+      const uint4 q = *reinterpret_cast<const uint4*>(src + 32 * c);
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    if ((sb >> e) & 1u) v[e] = -v[e];
-  }
-  // Stage h = 1 inside the thread, one rounding per sum or difference.
-#pragma unroll
-  for (int e = 0; e < E; e += 2) {
-    const float a = v[e], b = v[e + 1];
-    v[e] = a + b;
-    v[e + 1] = a - b;
-  }
-  // Stages h = 2 .. E/2: both members of a pair (e, e + 1) meet (e + h, e + 1 + h), in packed f32x2.
-#pragma unroll
-  for (int h = 2; h < E; h *= 2) {
-#pragma unroll
-    for (int e = 0; e < E; e += 2) {
-      if ((e & h) == 0) {
-        const uint64_t a = f2_pack(v[e], v[e + 1]), b = f2_pack(v[e + h], v[e + 1 + h]);
-        f2_unpack(f2_add(a, b), v[e], v[e + 1]);
-        f2_unpack(f2_add(a, f2_mul(b, f2_pack(-1.0f, -1.0f))), v[e + h], v[e + 1 + h]);
+      for (int i = 0; i < 4; ++i) {
+        v[8 * c + 2 * i] = __uint_as_float(w[i] << 16);
+        v[8 * c + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
       }
     }
   }
-  // The two stages across the row's four threads: the partner of element
-  // i = part*E + e is i ^ h, in part ^ (h / E) at the same e; the lower
-  // member keeps v + other, the upper other - v (one rounding each).
+}
+
+// One in-thread stage of the transform over the thread's list: pairs (e, e + h)
+// with bit h of e clear, taken two at a time in packed f32x2.
+template <int E, int H>
+__device__ __forceinline__ void quant_stage(float (&v)[E]) {
+  if constexpr (H == 1) {
+#pragma unroll
+    for (int e = 0; e < E; e += 2) {
+      const float a = v[e], b = v[e + 1];
+      v[e] = a + b;
+      v[e + 1] = a - b;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < E; e += 2) {
+      if ((e & H) == 0) {
+        const uint64_t a = f2_pack(v[e], v[e + 1]), b = f2_pack(v[e + H], v[e + 1 + H]);
+        f2_unpack(f2_add(a, b), v[e], v[e + 1]);
+        f2_unpack(f2_add(a, f2_mul(b, f2_pack(-1.0f, -1.0f))), v[e + H], v[e + 1 + H]);
+      }
+    }
+  }
+}
+
+// The signs and the unnormalised transform x H_d over the thread's E values
+// (the factor 1/sqrt(d) is applied by the caller).  sb[c] holds the 8 sign
+// bits of chunk c (bit j set: element j of the chunk is negated).
+template <int E>
+__device__ __forceinline__ void quant_rotate_row(int part, const uint32_t (&sb)[E / 8], float (&v)[E]) {
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    if ((sb[e / 8] >> (e % 8)) & 1u) v[e] = -v[e];
+  }
+  quant_stage<E, 1>(v);
+  quant_stage<E, 2>(v);
+  quant_stage<E, 4>(v);
+  // Half-widths 8 and 16: the partner of element i is i ^ h, in lane part ^ (h / 8)
+  // at the same position; the lower member keeps v + other, the upper other - v.
 #pragma unroll
   for (int hp = 1; hp < kQuantThreadsPerRow; hp *= 2) {
     const float sg = (part & hp) ? -1.0f : 1.0f;
@@ -136,108 +148,152 @@ __device__ __forceinline__ void quant_transform_row(const QuantParams& p, const 
       f2_unpack(f2_fma(f2_pack(v[e], v[e + 1]), sg2, f2_pack(o0, o1)), v[e], v[e + 1]);
     }
   }
+  // Half-widths 32 and 64: chunk bits of the thread's list (8 and 16 in it).
+  quant_stage<E, 8>(v);
+  if constexpr (E > 16) quant_stage<E, 16>(v);
 }
 
 // Stores E4M3(v * mul): mul = c / s, with c = float32(1/sqrt(d)) after a
 // rotation (else 1) and s the block's power-of-two descale, so that
-// v * mul = (v * c) / s exactly (s is a power of two).
+// v * mul = (v * c) / s exactly (s is a power of two).  Chunk c goes to row
+// bytes 32 c + 8 part .. + 7.
 template <int E>
-__device__ __forceinline__ void quant_store_row(const QuantParams& p, int z, int row, int part, const float (&v)[E],
-                                                float mul) {
-  uint4* dst = reinterpret_cast<uint4*>(p.xq + (static_cast<int64_t>(z) * p.N + row) * p.d + part * E);
+__device__ __forceinline__ void quant_store_row(uint8_t* dst_row, int part, const float (&v)[E], float mul) {
   const uint64_t m2 = f2_pack(mul, mul);
 #pragma unroll
-  for (int c = 0; c < E / 16; ++c) {
-    uint32_t w[4];
+  for (int c = 0; c < E / 8; ++c) {
+    uint32_t w[2];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = c * 16 + 4 * j;
+    for (int j = 0; j < 2; ++j) {
+      const int e = 8 * c + 4 * j;
       float a, b, cc, dd;
       f2_unpack(f2_mul(f2_pack(v[e], v[e + 1]), m2), a, b);
       f2_unpack(f2_mul(f2_pack(v[e + 2], v[e + 3]), m2), cc, dd);
       w[j] = cvt_e4m3x4(a, b, cc, dd);
     }
-    dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint2*>(dst_row + 32 * c + 8 * part) = make_uint2(w[0], w[1]);
   }
 }
 
-// MODE 0: scale per block of p.block_rows rows (one CTA per block, rows kept
-//         in registers between the amax and the cast).
-// MODE 1: per-slab pass 1 -- amax of the CTA's 128 rows, atomicMax into
+// Ring geometry of one launch: a stage holds one block of p.block_rows rows.
+__host__ __device__ inline int quant_stage_bytes(const QuantParams& p) {
+  return p.block_rows * p.d * (p.x_f32 ? 4 : 2);
+}
+__host__ __device__ inline int quant_stages(const QuantParams& p) {
+  const int n = kQuantStageBudget / quant_stage_bytes(p);
+  return n < 1 ? 1 : (n > kQuantMaxStages ? kQuantMaxStages : n);
+}
+
+// MODE 0: scale per block of p.block_rows rows (rows kept in registers
+//         between the amax and the cast).
+// MODE 1: per-slab pass 1 -- amax of each 128-row block, atomicMax into
 //         p.scales[z] (float bits of a value >= 0 order like integers).
 // MODE 2: per-slab pass 2 -- cast with the descale of the slab's amax.
+// The CTA walks the blocks u = blockIdx.x, blockIdx.x + gridDim.x, ... of the
+// Z * nblocks blocks (slab z = u / nblocks).
 template <int E, int MODE>
-__global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const QuantParams p, uint32_t* err_word) {
   constexpr int kPasses = 128 / kQuantRowsPerPass;  // rows per thread held in registers (block_rows <= 128)
-  __shared__ float warp_amax[kQuantWarps];
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ __align__(8) uint64_t full[kQuantMaxStages];
+  __shared__ float warp_amax[2][kQuantWarps];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int part = lane & (kQuantThreadsPerRow - 1);
   const int rsub = threadIdx.x / kQuantThreadsPerRow;  // 0..63
-  const int blk = blockIdx.x, z = blockIdx.y;
-  const int r0 = blk * p.block_rows;
-  const int rows = min(p.block_rows, p.N - r0);
-  // All of the thread's rows are fetched before any is transformed, so their
-  // loads are in flight together.
-  RowBits<E> raw[kPasses];
-#pragma unroll
-  for (int i = 0; i < kPasses; ++i) {
-    const int r = rsub + i * kQuantRowsPerPass;
-    if (r < rows) {
-      raw[i] = quant_fetch_row<E>(p, z, r0 + r, part);
-    } else {
-#pragma unroll
-      for (int j = 0; j < E / 4; ++j) raw[i].w[j] = make_uint4(0u, 0u, 0u, 0u);
-    }
+  const int row_bytes = p.d * (p.x_f32 ? 4 : 2);
+  const int stage_bytes = quant_stage_bytes(p);
+  const int stages = quant_stages(p);
+  const int nunits = p.Z * p.nblocks;
+  const uint8_t* xb = static_cast<const uint8_t*>(p.x);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
+    fence_mbar_init();
   }
-  // This thread's E sign bits: E = 32 is one whole word, E = 16 half of one.
-  uint32_t sb;
-  {
-    const int i0 = part * E;
-    const int wi = i0 >> 5;
-    sb = (wi == 0 ? p.sign_bits[0] : wi == 1 ? p.sign_bits[1] : wi == 2 ? p.sign_bits[2] : p.sign_bits[3]) >>
-         (i0 & 31);
+  __syncthreads();
+  // Copy of the CTA's local block k into stage k % stages (thread 0 only).
+  auto issue = [&](int k) {
+    const int u = blockIdx.x + k * gridDim.x;
+    if (u >= nunits) return;
+    const int z = u / p.nblocks, blk = u - z * p.nblocks;
+    const int r0 = blk * p.block_rows;
+    const uint32_t bytes = static_cast<uint32_t>(min(p.block_rows, p.N - r0) * row_bytes);
+    uint64_t* bar = &full[k % stages];
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load(ring + (k % stages) * stage_bytes, xb + (static_cast<int64_t>(z) * p.N + r0) * row_bytes, bytes, bar);
+  };
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < stages; ++k) issue(k);
   }
+
+  // This thread's sign bits: chunk c covers row elements 32 c + 8 part .. + 7.
+  uint32_t sb[E / 8];
+#pragma unroll
+  for (int c = 0; c < E / 8; ++c) sb[c] = (p.sign_bits[c] >> (8 * part)) & 0xFFu;
   // float32(1/sqrt(d)) after a rotation: applied to the block maximum here
   // (positive scaling is monotone, so max |v c| = max|v| c) and folded into
   // the cast's multiplier.
   const float cnorm = p.rotate ? ((E == 32) ? 0.08838834764831845f : 0.125f) : 1.0f;
-  float v[kPasses][E];
-  float amax = 0.0f;
+
+  int k = 0;
+  bool aborted = false;
+  for (int u = blockIdx.x; u < nunits; u += gridDim.x, ++k) {
+    const int z = u / p.nblocks, blk = u - z * p.nblocks;
+    const int r0 = blk * p.block_rows;
+    const int rows = min(p.block_rows, p.N - r0);
+    const bool ok = mbar_wait_bounded(&full[k % stages], (k / stages) & 1, err_word, kErrTimeoutLoad);
+    const uint8_t* stage = ring + (k % stages) * stage_bytes;
+    float v[kPasses][E];
+    float amax = 0.0f;
 #pragma unroll
-  for (int i = 0; i < kPasses; ++i) {
-    // Every lane transforms (rows past the block's end hold zeros), so the
-    // full-warp shuffles of the rotation always have all 32 lanes.
-    const int r = rsub + i * kQuantRowsPerPass;
-    quant_transform_row<E>(p, raw[i], part, sb, v[i]);
-    if (r < rows) {
+    for (int i = 0; i < kPasses; ++i) {
+      // Every lane transforms (rows past the block's end hold zeros), so the
+      // full-warp shuffles of the rotation always have all 32 lanes.
+      quant_read_row<E>(stage, row_bytes, rsub + i * kQuantRowsPerPass, ok ? rows : 0, part, p.x_f32, v[i]);
+      if (p.rotate) quant_rotate_row<E>(part, sb, v[i]);
 #pragma unroll
       for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(v[i][e]));
     }
-  }
-  amax *= cnorm;
-  int e;
-  if constexpr (MODE == 2) {
-    e = quant_scale_exponent(__uint_as_float(reinterpret_cast<const uint32_t*>(p.scales)[z]));
-  } else {
+    if constexpr (MODE != 2) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    if (lane == 0) warp_amax[warp] = amax;
-    __syncthreads();
-    float a = warp_amax[0];
-#pragma unroll
-    for (int w = 1; w < kQuantWarps; ++w) a = fmaxf(a, warp_amax[w]);
-    if constexpr (MODE == 1) {
-      if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned int*>(p.scales + z), __float_as_uint(a));
-      return;
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      if (lane == 0) warp_amax[k & 1][warp] = amax;
     }
-    e = quant_scale_exponent(a);
-    if (threadIdx.x == 0) p.scales[static_cast<int64_t>(z) * p.nblocks + blk] = ldexpf(1.0f, e);
-  }
-  const float mul = cnorm * ldexpf(1.0f, -e);  // c / s, exact (s a power of two)
+    // Every thread holds its rows: the stage goes back to the copy engine.
+    if (__syncthreads_or(!ok)) {
+      aborted = true;
+      break;
+    }
+    if (threadIdx.x == 0) issue(k + stages);
+    int e;
+    if constexpr (MODE == 2) {
+      e = quant_scale_exponent(__uint_as_float(reinterpret_cast<const uint32_t*>(p.scales)[z]));
+    } else {
+      float a = warp_amax[k & 1][0];
 #pragma unroll
-  for (int i = 0; i < kPasses; ++i) {
-    const int r = rsub + i * kQuantRowsPerPass;
-    if (r < rows) quant_store_row<E>(p, z, r0 + r, part, v[i], mul);
+      for (int w = 1; w < kQuantWarps; ++w) a = fmaxf(a, warp_amax[k & 1][w]);
+      a *= cnorm;
+      if constexpr (MODE == 1) {
+        if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned int*>(p.scales + z), __float_as_uint(a));
+        continue;
+      }
+      e = quant_scale_exponent(a);
+      if (threadIdx.x == 0) p.scales[static_cast<int64_t>(z) * p.nblocks + blk] = ldexpf(1.0f, e);
+    }
+    const float mul = cnorm * ldexpf(1.0f, -e);  // c / s, exact (s a power of two)
+#pragma unroll
+    for (int i = 0; i < kPasses; ++i) {
+      const int r = rsub + i * kQuantRowsPerPass;
+      if (r < rows) quant_store_row<E>(p.xq + (static_cast<int64_t>(z) * p.N + r0 + r) * p.d, part, v[i], mul);
+    }
+  }
+  // After a wait ran out: let the copies still in flight land before the CTA's
+  // shared memory is released (each wait again bounded).
+  if (threadIdx.x == 0 && aborted) {
+    for (int j = k; j < k + stages; ++j) {
+      if (blockIdx.x + j * gridDim.x >= nunits) break;
+      mbar_wait_bounded(&full[j % stages], (j / stages) & 1, err_word, kErrTimeoutLoad, 100000000ull);
+    }
   }
 }
 

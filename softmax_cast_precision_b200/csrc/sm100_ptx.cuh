@@ -19,6 +19,7 @@ enum : uint32_t {
   kErrTimeoutMMA = 1u << 1,   // waiting for an MMA commit
   kErrTimeoutQ = 1u << 2,     // waiting for the Q tile load
   kErrTimeoutPipe = 1u << 3,  // waiting on an internal pipeline barrier
+  kErrTimeoutLoad = 1u << 4,  // waiting for a bulk copy of input rows
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -123,6 +124,16 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(smem_dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Untiled bulk copy of `bytes` contiguous bytes from global to shared memory,
+// completing on `bar` (both addresses 16-byte aligned, bytes a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 

@@ -134,6 +134,7 @@ def _call_quantize(fp8, x=16, dtype=0, xq=16, scales=16, Z=2, N=300, d=128, bloc
     (dict(d=96), 2), (dict(d=256), 2), (dict(dtype=2), 1), (dict(block_rows=-1), 1), (dict(block_rows=129), 1),
     (dict(Z=-1), 1), (dict(N=-1), 1), (dict(x=0), 1), (dict(x=8), 1), (dict(xq=8), 1), (dict(scales=0), 1),
     (dict(scales=2), 1), (dict(Z=70000), 2), (dict(signs=[1.0] * 127 + [0.5]), 1),
+    (dict(Z=65535, N=20000, d=64, block_rows=1), 2),  # more than 2^30 blocks
     (dict(Z=0), 0), (dict(N=0), 0), (dict(N=0, x=0, xq=0), 0),
 ])
 def test_quantize_validation(fp8, kw, expected):
