@@ -24,7 +24,7 @@ runs the scaled forward pass, which rotates the output back.
 path) with E4M3 V: the P-cast summary's kernel-faithful setting.
 
 --path decode times the split-KV decode pass (B=32, H=32, Hkv=8, N=32768,
-one query row per head, 16-tile splits) against the HBM roofline.
+one query row per head, 32-tile splits) against the HBM roofline.
 
 --path bwd times the backward pass of the 32K prefill (dQ, dK, dV from the
 forward's inputs, O, lse and a bfloat16 dO).
@@ -565,7 +565,7 @@ def run_bf16qk(args, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
-DECODE_SHAPE = dict(B=32, H=32, Hkv=8, N=32768, split_tiles=16)
+DECODE_SHAPE = dict(B=32, H=32, Hkv=8, N=32768, split_tiles=32)
 DECODE_METRIC = "FP8 split-KV decode GB/s of K/V read (HBM roofline)"
 
 

@@ -50,12 +50,11 @@ struct DecodeParams {
 };
 
 constexpr int kTcN = 16;         // query heads padded to the MMA's N
-constexpr int kDecodeStages = 2;  // K/V ring: tile i + 1 loads while tile i is consumed
 
 struct DecodeLayout {
-  static constexpr int OFF_K = 0;                                 // kDecodeStages x 16 KB (TMA, 128-byte swizzle)
-  static constexpr int OFF_V = kDecodeStages * 16384;             // kDecodeStages x 16 KB
-  static constexpr int OFF_Q = 2 * kDecodeStages * 16384;         // Q: 16 rows x 128 B, K-major (B of S^T)
+  static constexpr int OFF_K = 0;                       // 2 stages x 16 KB (TMA, 128-byte swizzle)
+  static constexpr int OFF_V = 2 * 16384;               // 2 stages x 16 KB
+  static constexpr int OFF_Q = 4 * 16384;               // Q: 16 rows x 128 B, K-major (B of S^T)
   static constexpr int OFF_P = OFF_Q + 2048;            // P^: 16 rows x 128 keys, K-major (B of O^T)
   static constexpr int OFF_RED = OFF_P + 2048;          // float [2][4 warps][16]: maxima, sums
   static constexpr int OFF_BAR = OFF_RED + 2 * 4 * kTcN * 4;
@@ -72,11 +71,12 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
   float* sMax = reinterpret_cast<float*>(base + L::OFF_RED);  // [4][16]
   float* sSum = sMax + 4 * kTcN;                               // [4][16]
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
-  uint64_t* bar_kv = bars + 0;               // per stage: K and V of a tile landed
-  uint64_t* bar_s = bars + kDecodeStages;     // S^T of the next tile computed
-  uint64_t* bar_o = bars + kDecodeStages + 1; // O^T += P^ V of this tile complete
-  uint64_t* bar_drain = bars + kDecodeStages + 2;  // every product issued so far complete (abort path)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kDecodeStages + 3);
+  uint64_t* bar_k = bars + 0;      // per stage: K of a tile landed
+  uint64_t* bar_v = bars + 2;      // per stage: V of a tile landed
+  uint64_t* bar_s = bars + 4;      // S^T of the next tile computed
+  uint64_t* bar_o = bars + 5;      // O^T += P^ V of this tile complete
+  uint64_t* bar_drain = bars + 6;  // every product issued so far complete (abort path)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
 
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int split = blockIdx.x, zkv = blockIdx.y;  // zkv = b * Hkv + hkv
@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
   auto tile_of = [&](int i) { return tile0 + (p.reverse ? nt - 1 - i : i); };
 
   if (t == 0) {
-    for (int i = 0; i < kDecodeStages + 3; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < 7; ++i) mbar_init(bars + i, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
@@ -122,37 +122,51 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
   const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t tO = tmem + 32;  // O^T: columns 32 .. 47; S^T buffers at 0 .. 15 and 16 .. 31
 
-  int issued = 0, landed = 0;     // thread 0: tiles whose loads were issued / waited for
-  auto issue_tile = [&](int i) {  // K and V of the split's i-th tile into stage i % kDecodeStages
-    const int st = i % kDecodeStages;
-    issued = i + 1;
-    mbar_arrive_expect_tx(bar_kv + st, 2 * 16384);
-    tma_load_3d(base + L::OFF_K + st * 16384, &tm_k, bar_kv + st, 0, tile_of(i) * 128, zkv);
-    tma_load_3d(base + L::OFF_V + st * 16384, &tm_v, bar_kv + st, 0, tile_of(i) * 128, zkv);
+  // Thread 0 issues the copies and the products.  K and V of tile i go to
+  // stage i % 2 on barriers of their own: a K stage is free once the S^T it
+  // fed has completed, so K runs two tiles ahead; a V stage is free once the
+  // P^ V it fed has completed.
+  int k_issued = 0, k_landed = 0, v_issued = 0, v_landed = 0;  // thread 0: tiles issued / waited for
+  auto issue_k = [&](int i) {
+    k_issued = i + 1;
+    mbar_arrive_expect_tx(bar_k + (i & 1), 16384);
+    tma_load_3d(base + L::OFF_K + (i & 1) * 16384, &tm_k, bar_k + (i & 1), 0, tile_of(i) * 128, zkv);
+  };
+  auto issue_v = [&](int i) {
+    v_issued = i + 1;
+    mbar_arrive_expect_tx(bar_v + (i & 1), 16384);
+    tma_load_3d(base + L::OFF_V + (i & 1) * 16384, &tm_v, bar_v + (i & 1), 0, tile_of(i) * 128, zkv);
   };
   constexpr uint32_t idesc_s = idesc_e4m3_f32(128, kTcN, false, false);
   constexpr uint32_t idesc_o = idesc_e4m3_f32(128, kTcN, true, false);  // A = V^T read MN-major
   const uint64_t dQ = smem_desc(smem_u32(base + L::OFF_Q), 16, 1024, 2);
   const uint64_t dP = smem_desc(smem_u32(base + L::OFF_P), 16, 1024, 2);
-  auto issue_s = [&](int i) {  // S^T of tile i into TMEM buffer i % 2 (its K must have landed)
-    const uint64_t dK = smem_desc(smem_u32(base + L::OFF_K + (i % kDecodeStages) * 16384), 16, 1024, 2);
+  // S^T of tile i into TMEM buffer i % 2, once its K has landed.
+  auto issue_s = [&](int i) -> bool {
+    if (!mbar_wait_bounded(bar_k + (i & 1), (i >> 1) & 1, err_word, kErrTimeoutKV)) return false;
+    k_landed = i + 1;
+    tc_fence_after();
+    const uint64_t dK = smem_desc(smem_u32(base + L::OFF_K + (i & 1) * 16384), 16, 1024, 2);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tmem + (i & 1) * 16, dK + 2 * kk, dQ + 2 * kk, idesc_s, kk > 0);
     mma_commit(bar_s);
+    return true;
   };
 
   bool fail = false;
   if (t == 0) {
-    for (int i = 0; i < kDecodeStages && i < nt; ++i) issue_tile(i);
-    if (mbar_wait_bounded(bar_kv, 0, err_word, kErrTimeoutKV)) {
-      landed = 1;
-      tc_fence_after();
-      issue_s(0);
-    } else {
-      fail = true;
+    issue_k(0);
+    issue_v(0);
+    if (nt > 1) {
+      issue_k(1);
+      issue_v(1);
     }
+    fail = !issue_s(0);
   }
 
+  // m: running maximum of each query head's logits (uniform over the CTA);
+  // l: this thread's share of l * S (its keys' unquantised P * S), summed
+  // over the CTA once at the end.
   float m[kTcN], l[kTcN];
 #pragma unroll
   for (int g = 0; g < kTcN; ++g) m[g] = -INFINITY, l[g] = 0.0f;
@@ -165,58 +179,49 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
     // This tile's logits.
     if (!mbar_wait_bounded(bar_s, i & 1, err_word, kErrTimeoutMMA)) fail = true;
     tc_fence_after();
+    // S^T(i) is complete, so K stage i % 2 is free for tile i + 2.
+    if (t == 0 && !fail && i + 2 < nt) issue_k(i + 2);
     uint32_t rs[16];
     tmem_ld16(tmem + (i & 1) * 16 + lane_off, rs);
     tmem_wait_ld();
     float s[kTcN];
 #pragma unroll
     for (int g = 0; g < kTcN; ++g) s[g] = __uint_as_float(rs[g]);
-    // Tile maximum of every query head: warp, then the four warps.
+    // Tile maximum of every query head: one warp reduction, then the four warps.
 #pragma unroll
     for (int g = 0; g < kTcN; ++g) {
       if (g < G) {
-        float x = valid ? s[g] : -INFINITY;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+        const float x = warp_max_f32(valid ? s[g] : -INFINITY);
         if (lane == 0) sMax[warp * kTcN + g] = x;
       }
     }
     // The previous P^ V must be complete before P^ and O^T are touched; its
-    // stage is then free for tile i - 1 + kDecodeStages.
+    // V stage is then free for tile i + 1.
     if (i > 0) {
       if (!mbar_wait_bounded(bar_o, (i - 1) & 1, err_word, kErrTimeoutMMA)) fail = true;
       tc_fence_after();
-      if (t == 0 && !fail && i - 1 + kDecodeStages < nt) issue_tile(i - 1 + kDecodeStages);
+      if (t == 0 && !fail && i + 1 < nt) issue_v(i + 1);
     }
     abort = __syncthreads_or(fail) != 0;
     if (abort) break;
+    const float* tm = sMax;
     float alpha[kTcN];
     bool any_rescale = false;
 #pragma unroll
     for (int g = 0; g < kTcN; ++g) {
       alpha[g] = 1.0f;
       if (g < G) {
-        const float tmax = fmaxf(fmaxf(sMax[g], sMax[kTcN + g]), fmaxf(sMax[2 * kTcN + g], sMax[3 * kTcN + g]));
+        const float tmax = fmaxf(fmaxf(tm[g], tm[kTcN + g]), fmaxf(tm[2 * kTcN + g], tm[3 * kTcN + g]));
         const float m_new = fmaxf(m[g], tmax * c);
         alpha[g] = (m_new == m[g]) ? 1.0f : ex2_approx(m[g] - m_new);
         any_rescale |= alpha[g] != 1.0f;
         m[g] = m_new;
         // P * S for key t: the scale enters the exponent; masked keys give 0.
         const float ps = valid ? ex2_approx(fmaf(s[g], c, p.log2_p_scale - m_new)) : 0.0f;
-        s[g] = ps;
+        l[g] = l[g] * alpha[g] + ps;
         const uint32_t code = cvt_e4m3x2(ps, 0.0f) & 0xFFu;
         const uint32_t off = g * 128 + ((((t >> 4) ^ (g & 7))) << 4) + (t & 15);
         asm volatile("st.shared.u8 [%0], %1;" ::"r"(smem_u32(base + L::OFF_P) + off), "r"(code) : "memory");
-      }
-    }
-    // Row sums of the unquantised P * S.
-#pragma unroll
-    for (int g = 0; g < kTcN; ++g) {
-      if (g < G) {
-        float x = s[g];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-        if (lane == 0) sSum[warp * kTcN + g] = x;
       }
     }
     // O^T *= alpha per query head (column), when any maximum grew; every
@@ -233,38 +238,37 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-#pragma unroll
-    for (int g = 0; g < kTcN; ++g) {
-      if (g < G) {
-        const float tsum = (sSum[g] + sSum[kTcN + g]) + (sSum[2 * kTcN + g] + sSum[3 * kTcN + g]);
-        l[g] = l[g] * alpha[g] + tsum;  // l * S
-      }
-    }
     if (t == 0) {
-      tc_fence_after();
-      // O^T += V^T P^^T: V stage i % kDecodeStages read MN-major (32 keys = 32 rows of 128 B per step).
-      const uint64_t dV = smem_desc(smem_u32(base + L::OFF_V + (i % kDecodeStages) * 16384), 16384, 1024, 2);
+      // O^T += V^T P^^T once V(i) has landed: V stage i % 2 read MN-major (32 keys = 32 rows of 128 B per step).
+      if (mbar_wait_bounded(bar_v + (i & 1), (i >> 1) & 1, err_word, kErrTimeoutKV)) {
+        v_landed = i + 1;
+        tc_fence_after();
+        const uint64_t dV = smem_desc(smem_u32(base + L::OFF_V + (i & 1) * 16384), 16384, 1024, 2);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tO, dV + 256 * kk, dP + 2 * kk, idesc_o, (i > 0) || (kk > 0));
-      mma_commit(bar_o);
-      if (i + 1 < nt) {
-        const int st = (i + 1) % kDecodeStages;
-        if (mbar_wait_bounded(bar_kv + st, ((i + 1) / kDecodeStages) & 1, err_word, kErrTimeoutKV)) {
-          landed = i + 2;
-          tc_fence_after();
-          issue_s(i + 1);
-        } else {
-          fail = true;
-        }
+        for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tO, dV + 256 * kk, dP + 2 * kk, idesc_o, (i > 0) || (kk > 0));
+        mma_commit(bar_o);
+        if (i + 1 < nt && !issue_s(i + 1)) fail = true;
+      } else {
+        fail = true;
       }
     }
-    // The sums are read before the next tile rewrites them: the next
-    // tile's first barrier comes after its maxima, and the sums after it.
+    // Every thread read this tile's maxima before the barrier above, so the
+    // next tile may overwrite them.
   }
   abort = __syncthreads_or(fail || abort) != 0;
   if (!abort && nt > 0) {
     if (!mbar_wait_bounded(bar_o, (nt - 1) & 1, err_word, kErrTimeoutMMA)) abort = true;
     tc_fence_after();
+  }
+  // l * S of each query head: the threads' shares, summed over the warp, then the warps.
+#pragma unroll
+  for (int g = 0; g < kTcN; ++g) {
+    if (g < G) {
+      float x = l[g];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+      if (lane == 0) sSum[warp * kTcN + g] = x;
+    }
   }
   abort = __syncthreads_or(abort) != 0;
   if (!abort) {
@@ -279,7 +283,7 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
         dst[t] = __uint_as_float(o[g]);
         if (t == 0) {
           dst[128] = m[g];
-          dst[129] = l[g];
+          dst[129] = (sSum[g] + sSum[kTcN + g]) + (sSum[2 * kTcN + g] + sSum[3 * kTcN + g]);
         }
       }
     }
@@ -290,8 +294,10 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const __grid_constant
     // bounded).
     mma_commit(bar_drain);
     mbar_wait_bounded(bar_drain, 0, err_word, kErrTimeoutMMA, 100000000ull);
-    for (int j = landed; j < issued; ++j)
-      mbar_wait_bounded(bar_kv + j % kDecodeStages, (j / kDecodeStages) & 1, err_word, kErrTimeoutKV, 100000000ull);
+    for (int j = k_landed; j < k_issued; ++j)
+      mbar_wait_bounded(bar_k + (j & 1), (j >> 1) & 1, err_word, kErrTimeoutKV, 100000000ull);
+    for (int j = v_landed; j < v_issued; ++j)
+      mbar_wait_bounded(bar_v + (j & 1), (j >> 1) & 1, err_word, kErrTimeoutKV, 100000000ull);
   }
   tc_fence_before();
   __syncthreads();
