@@ -52,6 +52,7 @@ constexpr int kQuantWarps = 8;
 constexpr int kQuantThreadsPerRow = 4;
 constexpr int kQuantRowsPerPass = kQuantWarps * 32 / kQuantThreadsPerRow;  // 64
 constexpr int kQuantMaxStages = 8;
+constexpr int kQuantMaxChunks = 4;  // 8-element chunks per thread at d = 128
 constexpr int kQuantStageBudget = 96 * 1024;  // shared bytes of the ring (two CTAs per SM)
 
 // Binary exponent e of the descale s = 2^e of a block whose largest
@@ -69,7 +70,7 @@ __device__ __forceinline__ int quant_scale_exponent(float amax) {
 // Rows past the block's end read as zeros.
 template <int E>
 __device__ __forceinline__ void quant_read_row(const uint8_t* stage, int row_bytes, int r, int rows, int part,
-                                               int x_f32, float (&v)[E]) {
+                                               int x_f32, const uint4* sign_masks, float (&v)[E]) {
   if (r >= rows) {
 #pragma unroll
     for (int e = 0; e < E; ++e) v[e] = 0.0f;
@@ -90,7 +91,9 @@ __device__ __forceinline__ void quant_read_row(const uint8_t* stage, int row_byt
 #pragma unroll
     for (int c = 0; c < E / 8; ++c) {
       const uint4 q = *reinterpret_cast<const uint4*>(src + 32 * c);
-      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+      // With a rotation, the signs flip the bfloat16 sign bits (bits 15 and 31 of each word).
+      const uint4 sm = sign_masks ? sign_masks[c * kQuantThreadsPerRow + part] : make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t w[4] = {q.x ^ sm.x, q.y ^ sm.y, q.z ^ sm.z, q.w ^ sm.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         v[8 * c + 2 * i] = __uint_as_float(w[i] << 16);
@@ -117,7 +120,7 @@ __device__ __forceinline__ void quant_stage(float (&v)[E]) {
       if ((e & H) == 0) {
         const uint64_t a = f2_pack(v[e], v[e + 1]), b = f2_pack(v[e + H], v[e + 1 + H]);
         f2_unpack(f2_add(a, b), v[e], v[e + 1]);
-        f2_unpack(f2_add(a, f2_mul(b, f2_pack(-1.0f, -1.0f))), v[e + H], v[e + 1 + H]);
+        f2_unpack(f2_fma(b, f2_pack(-1.0f, -1.0f), a), v[e + H], v[e + 1 + H]);  // a - b, one rounding
       }
     }
   }
@@ -127,10 +130,13 @@ __device__ __forceinline__ void quant_stage(float (&v)[E]) {
 // (the factor 1/sqrt(d) is applied by the caller).  sb[c] holds the 8 sign
 // bits of chunk c (bit j set: element j of the chunk is negated).
 template <int E>
-__device__ __forceinline__ void quant_rotate_row(int part, const uint32_t (&sb)[E / 8], float (&v)[E]) {
+__device__ __forceinline__ void quant_rotate_row(int part, const uint32_t (&sb)[E / 8], bool signs_applied,
+                                                 float (&v)[E]) {
+  if (!signs_applied) {
 #pragma unroll
-  for (int e = 0; e < E; ++e) {
-    if ((sb[e / 8] >> (e % 8)) & 1u) v[e] = -v[e];
+    for (int e = 0; e < E; ++e) {
+      if ((sb[e / 8] >> (e % 8)) & 1u) v[e] = -v[e];
+    }
   }
   quant_stage<E, 1>(v);
   quant_stage<E, 2>(v);
@@ -197,6 +203,9 @@ __global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const Qua
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ __align__(8) uint64_t full[kQuantMaxStages];
   __shared__ float warp_amax[2][kQuantWarps];
+  // bfloat16 inputs with a rotation: XOR masks of the signs, per (chunk, part),
+  // for the four 32-bit words (two elements each) of a chunk.
+  __shared__ uint4 sign_masks[kQuantMaxChunks * kQuantThreadsPerRow];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int part = lane & (kQuantThreadsPerRow - 1);
   const int rsub = threadIdx.x / kQuantThreadsPerRow;  // 0..63
@@ -209,6 +218,17 @@ __global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const Qua
   if (threadIdx.x == 0) {
     for (int s = 0; s < stages; ++s) mbar_init(&full[s], 1);
     fence_mbar_init();
+  }
+  const bool word_signs = p.rotate && !p.x_f32;
+  if (word_signs && threadIdx.x < (E / 8) * kQuantThreadsPerRow) {
+    const int c = threadIdx.x / kQuantThreadsPerRow, pt = threadIdx.x % kQuantThreadsPerRow;
+    // (no run-time index into the parameter array, which would copy it to local memory)
+    const uint32_t word = c == 0 ? p.sign_bits[0] : c == 1 ? p.sign_bits[1] : c == 2 ? p.sign_bits[2] : p.sign_bits[3];
+    const uint32_t x = (word >> (8 * pt)) & 0xFFu;  // elements 32 c + 8 pt + j, bit j
+    uint32_t m[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m[j] = (((x >> (2 * j)) & 1u) << 15) | (((x >> (2 * j + 1)) & 1u) << 31);
+    sign_masks[threadIdx.x] = make_uint4(m[0], m[1], m[2], m[3]);
   }
   __syncthreads();
   // Copy of the CTA's local block k into stage k % stages (thread 0 only).
@@ -249,8 +269,9 @@ __global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const Qua
     for (int i = 0; i < kPasses; ++i) {
       // Every lane transforms (rows past the block's end hold zeros), so the
       // full-warp shuffles of the rotation always have all 32 lanes.
-      quant_read_row<E>(stage, row_bytes, rsub + i * kQuantRowsPerPass, ok ? rows : 0, part, p.x_f32, v[i]);
-      if (p.rotate) quant_rotate_row<E>(part, sb, v[i]);
+      quant_read_row<E>(stage, row_bytes, rsub + i * kQuantRowsPerPass, ok ? rows : 0, part, p.x_f32,
+                        word_signs ? sign_masks : nullptr, v[i]);
+      if (p.rotate) quant_rotate_row<E>(part, sb, word_signs, v[i]);
 #pragma unroll
       for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(v[i][e]));
     }
