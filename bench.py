@@ -118,8 +118,9 @@ def kernel_source_hash() -> str:
             h.update(name.encode() + _strip_comments(fh.read()).encode())
     with open(os.path.join(csrc, "api.cu"), encoding="utf-8") as fh:
         api = fh.read()
-    m = re.search(r"\nint launch_v2\(.*?\n}\n", api, re.S)
-    h.update(_strip_comments(m.group(0) if m else api).encode())
+    for fn in ("launch_v2_on", "launch_v2"):
+        m = re.search(r"\nint " + fn + r"\(.*?\n}\n", api, re.S)
+        h.update(_strip_comments(m.group(0) if m else api).encode())
     return h.hexdigest()[:16]
 
 
@@ -1132,7 +1133,7 @@ def main():
                                     "frac_at_kernel_clock = achieved / (peak x kernel MHz / peak MHz)")},
         "e2e": {"value": aggregate_throughput(flops, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-                "how": "fwd_host with pinned host buffers, copies overlapped piece by piece; CUDA events"},
+                "how": "fp8attn_fwd_host with pinned host buffers: one persistent pass over pieces copied in and out on two copy streams; CUDA events"},
         "clocks": clocks,
         "mse_vs_fp64": {"value": mse, "rows": "256 evenly spaced query rows of each head",
                         "reference": "PyTorch float64 softmax(QK^T/sqrt(d))V on the same E4M3 inputs"},

@@ -240,6 +240,52 @@ int fp8attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, fl
                         int B, int H, int Hkv, int N, int d, int causal,
                         float p_scale, int kv_order, void* stream);
 
+/*
+ * The forward pass of fp8attn_fwd on inputs and outputs in HOST memory, with
+ * the host<->device copies overlapped with the computation ("P-Cast
+ * Precision in FP8 Attention", technical summary, section 1, for what is
+ * computed; the overlap is this library's).
+ *
+ * q_host, k_host, v_host (E4M3 bytes), o_host (bfloat16) and lse_host
+ * (float32, or NULL) have the layouts of fp8attn_fwd and should be pinned
+ * (cudaHostAlloc / cudaHostRegister) for the copies to overlap; pageable
+ * memory works, but its copies then run one after another.  q_dev, k_dev,
+ * v_dev, o_dev and lse_dev (NULL exactly when lse_host is NULL) are
+ * caller-owned device buffers of the same sizes, used as staging (16-byte
+ * aligned; lse_dev 4-byte aligned); their contents afterwards are those of
+ * an fp8attn_fwd call on them.
+ *
+ * The problem is cut into `pieces` (1..16; 0 picks 12) pieces of whole
+ * (batch, kv head) slabs with their query heads.  Piece c's inputs are copied
+ * on a copy stream of the library, which then sets a ready word; one
+ * persistent kernel on `stream` processes the pieces in order, its producer
+ * waiting for each piece's ready word; as the last query tile of a piece is
+ * stored the kernel raises the piece's flag, and a second copy stream copies
+ * that piece's outputs back as soon as the flag is up.  The copy streams are
+ * non-blocking streams the library creates once per device; the work on them
+ * is joined back into `stream` before the call's later work.  The ready
+ * words, flags and work-unit counter of a call sit in a 256-byte block of a
+ * ring of eight that the library allocates once per device (stream memory
+ * operations cannot address pool allocations); a block is reused only after
+ * the stream of its previous call has passed that call's end.  Calls from
+ * several host threads on one device must be ordered by the caller.
+ * With d = 64 or pieces = 1 the copies in, the pass and the copies out simply
+ * run in order on `stream`.
+ *
+ * Asynchronous like fp8attn_fwd: the outputs are on the host once `stream`
+ * has reached this point.  If a device wait runs out, the kernel still
+ * raises every flag (so no copy stream waits for good), the outputs are
+ * undefined, and fp8attn_check_error() returns FP8ATTN_ERR_TIMEOUT.
+ * Returns FP8ATTN_ERR_INVALID_ARG for a NULL host pointer, pieces outside
+ * 0..16 or the checks of fp8attn_fwd (on the device buffers);
+ * FP8ATTN_ERR_UNSUPPORTED if the driver has no stream memory operations.
+ */
+int fp8attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                     void* o_host, float* lse_host,
+                     void* q_dev, void* k_dev, void* v_dev, void* o_dev, float* lse_dev,
+                     int B, int H, int Hkv, int N, int d, int causal,
+                     float p_scale, int kv_order, int pieces, void* stream);
+
 /* KV block size B_c the kernels use for head dimension d (0 if d is
  * unsupported).  The query block is always 128 rows. */
 int fp8attn_kv_tile(int d);

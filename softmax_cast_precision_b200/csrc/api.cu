@@ -159,9 +159,11 @@ int num_sms() {
   return n;
 }
 
-// Persistent warp-specialised kernel (d = 128): one CTA per SM.
+// Persistent warp-specialised kernel (d = 128): one CTA per SM.  `sched`
+// is the work-unit counter, already zero on `stream`; p.stream_flags (if
+// set) and p.heads_per_piece describe a streamed call.
 template <bool COUNT, bool SCALED = false, bool QK16 = false>
-int launch_v2(const void* q, const void* k, const void* v, FwdParams p, cudaStream_t stream) {
+int launch_v2_on(const void* q, const void* k, const void* v, FwdParams p, cudaStream_t stream, unsigned int* sched) {
   using C = V2Config;
   constexpr int kSmem = V2Layout<QK16>::SMEM_BYTES;
   CUtensorMap tq, tk, tv;
@@ -200,20 +202,27 @@ int launch_v2(const void* q, const void* k, const void* v, FwdParams p, cudaStre
   int gh = (2 * grid + num_pairs - 1) / num_pairs;
   while (gh > 1 && ((gh + p.h_per_kv - 1) / p.h_per_kv + 1) * kv_head_bytes > (48ll << 20)) --gh;
   p.group_heads = gh < 1 ? 1 : (gh > p.B * p.H ? p.B * p.H : gh);
-  // Work units are claimed from a counter that must be zero at launch; it
-  // lives in a 256-byte block from the library's stream-ordered pool for the
-  // duration of this call, so concurrent calls on other streams never share it.
+  // A streamed call needs the units in piece order: whole groups per piece.
+  if (p.stream_flags != nullptr)
+    while (p.heads_per_piece % p.group_heads != 0) --p.group_heads;
+  p.sched = sched;
+  kern<<<grid, C::THREADS, kSmem, stream>>>(tq, tk, tv, p, err_word);
+  return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
+}
+
+// The same with its work-unit counter in a 256-byte block from the library's
+// stream-ordered pool for the duration of the call, so that concurrent calls
+// on other streams never share it.
+template <bool COUNT, bool SCALED = false, bool QK16 = false>
+int launch_v2(const void* q, const void* k, const void* v, FwdParams p, cudaStream_t stream) {
   void* sched = nullptr;
   cudaMemPool_t pool = sched_pool();
   if (!pool || cudaMallocFromPoolAsync(&sched, 256, pool, stream) != cudaSuccess) return FP8ATTN_ERR_CUDA;
   int status = FP8ATTN_OK;
-  if (cudaMemsetAsync(sched, 0, sizeof(unsigned int), stream) != cudaSuccess) {
+  if (cudaMemsetAsync(sched, 0, sizeof(unsigned int), stream) != cudaSuccess)
     status = FP8ATTN_ERR_CUDA;
-  } else {
-    p.sched = static_cast<unsigned int*>(sched);
-    kern<<<grid, C::THREADS, kSmem, stream>>>(tq, tk, tv, p, err_word);
-    if (cudaGetLastError() != cudaSuccess) status = FP8ATTN_ERR_CUDA;
-  }
+  else
+    status = launch_v2_on<COUNT, SCALED, QK16>(q, k, v, p, stream, static_cast<unsigned int*>(sched));
   if (cudaFreeAsync(sched, stream) != cudaSuccess) status = FP8ATTN_ERR_CUDA;
   return status;
 }
@@ -326,8 +335,169 @@ int launch_v2_noalloc(const void* q, const void* k, const void* v, FwdParams p, 
   return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
 }
 
+
+// ---- streamed host entry point (fp8attn_fwd_host) ----
+
+using StreamValueFn = CUresult (*)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
+
+StreamValueFn get_stream_value_fn(const char* name) {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion(name, &fn, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<StreamValueFn>(fn);
+}
+
+// Per-device copy streams, fork/join events and flag blocks of
+// fp8attn_fwd_host, made once.  The streams are non-blocking, so that they
+// never wait for the legacy default stream on which the kernel may be
+// running.  Stream memory operations reject stream-ordered (pool)
+// allocations, so the 256-byte blocks holding a call's work-unit counter,
+// ready words and flags come from one cudaMalloc: a ring of kHostBlocks, each
+// handed to a new call only after the stream of its previous call has passed
+// the event recorded at that call's end.
+constexpr int kHostBlocks = 8;
+struct HostStreams {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t fork = nullptr, in_done = nullptr, out_done = nullptr;
+  cudaEvent_t block_free[kHostBlocks] = {};
+  unsigned int* blocks = nullptr;  // kHostBlocks x 64 words
+  int next = 0;
+  StreamValueFn write32 = nullptr, wait32 = nullptr;
+  bool ready = false;
+};
+
+int host_streams(HostStreams** out) {
+  static HostStreams devs[64];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  HostStreams& h = devs[dev];
+  if (!h.ready) {
+    h.write32 = get_stream_value_fn("cuStreamWriteValue32");
+    h.wait32 = get_stream_value_fn("cuStreamWaitValue32");
+    if (!h.write32 || !h.wait32) return FP8ATTN_ERR_UNSUPPORTED;
+    if (cudaStreamCreateWithFlags(&h.in, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&h.out, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h.in_done, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&h.out_done, cudaEventDisableTiming) != cudaSuccess ||
+        cudaMalloc(reinterpret_cast<void**>(&h.blocks), kHostBlocks * 256) != cudaSuccess)
+      return FP8ATTN_ERR_CUDA;
+    for (int i = 0; i < kHostBlocks; ++i)
+      if (cudaEventCreateWithFlags(&h.block_free[i], cudaEventDisableTiming) != cudaSuccess) return FP8ATTN_ERR_CUDA;
+    h.ready = true;
+  }
+  *out = &h;
+  return FP8ATTN_OK;
+}
+
+// Takes the next flag block of the ring (its previous call's end is passed
+// on `s` before the block is touched); returns its index.
+int take_host_block(HostStreams* h, cudaStream_t s) {
+  static std::mutex mu;
+  int slot;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    slot = h->next;
+    h->next = (h->next + 1) % kHostBlocks;
+  }
+  return cudaStreamWaitEvent(s, h->block_free[slot], 0) == cudaSuccess ? slot : -1;
+}
+
 }  // namespace
 }  // namespace fp8attn
+
+extern "C" int fp8attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                                float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev, float* lse_dev,
+                                int B, int H, int Hkv, int N, int d, int causal, float p_scale, int kv_order,
+                                int pieces, void* stream) {
+  using namespace fp8attn;
+  int st = validate(q_dev, k_dev, v_dev, B, H, Hkv, N, d, p_scale, kv_order);
+  if (st != FP8ATTN_OK) return st;
+  if (pieces < 0 || pieces > kMaxPieces) return FP8ATTN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B) * H * N == 0) return FP8ATTN_OK;
+  if (!q_host || !k_host || !v_host || !o_host || !o_dev || !aligned16(o_dev) || (lse_host == nullptr) != (lse_dev == nullptr) ||
+      (lse_dev && (reinterpret_cast<uintptr_t>(lse_dev) & 3u)))
+    return FP8ATTN_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t row = static_cast<size_t>(N) * d;  // elements of one (b, h) slab
+  const size_t zq = static_cast<size_t>(B) * H, zkv = static_cast<size_t>(B) * Hkv;
+  auto h2d = [&](void* dst, const void* src, size_t bytes, cudaStream_t cs) {
+    return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyHostToDevice, cs) == cudaSuccess;
+  };
+  auto d2h = [&](void* dst, const void* src, size_t bytes, cudaStream_t cs) {
+    return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToHost, cs) == cudaSuccess;
+  };
+  FwdParams p = base_params(B, H, Hkv, N, causal, p_scale, kv_order);
+  p.o = o_dev;
+  p.lse = lse_dev;
+  if (d != 128 || pieces == 1) {
+    // One piece: copies in, the pass, copies out, in order on the stream.
+    if (!h2d(q_dev, q_host, zq * row, s) || !h2d(k_dev, k_host, zkv * row, s) || !h2d(v_dev, v_host, zkv * row, s))
+      return FP8ATTN_ERR_CUDA;
+    st = d == 128 ? launch_v2<false>(q_dev, k_dev, v_dev, p, s) : launch<64, false>(q_dev, k_dev, v_dev, p, s);
+    if (st != FP8ATTN_OK) return st;
+    if (!d2h(o_host, o_dev, zq * row * 2, s) || (lse_dev && !d2h(lse_host, lse_dev, zq * N * sizeof(float), s)))
+      return FP8ATTN_ERR_CUDA;
+    return FP8ATTN_OK;
+  }
+  HostStreams* hs = nullptr;
+  st = host_streams(&hs);
+  if (st != FP8ATTN_OK) return st;
+  // Pieces of whole (b, kv head) slabs with their query heads.
+  const int want = pieces == 0 ? 12 : pieces;
+  const int kv_per_piece = static_cast<int>((zkv + want - 1) / want);
+  const int n_pieces = static_cast<int>((zkv + kv_per_piece - 1) / kv_per_piece);
+  const int rep = H / Hkv;
+  p.heads_per_piece = kv_per_piece * rep;
+  // The 256-byte block holds the work-unit counter (word 0) and the piece words.
+  const int slot = take_host_block(hs, s);
+  if (slot < 0) return FP8ATTN_ERR_CUDA;
+  unsigned int* flags = hs->blocks + 64 * slot;
+  const CUdeviceptr fl = reinterpret_cast<CUdeviceptr>(flags);
+  p.stream_flags = flags;
+  bool ok = cudaMemsetAsync(flags, 0, 256, s) == cudaSuccess && cudaEventRecord(hs->fork, s) == cudaSuccess &&
+            cudaStreamWaitEvent(hs->in, hs->fork, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(hs->out, hs->fork, 0) == cudaSuccess;
+  // Copies in: each piece, then its ready word.
+  for (int c = 0; ok && c < n_pieces; ++c) {
+    const size_t k0 = static_cast<size_t>(c) * kv_per_piece;
+    const size_t nk = std::min<size_t>(kv_per_piece, zkv - k0);
+    const size_t q0 = k0 * rep, nq = nk * rep;
+    ok = h2d(static_cast<uint8_t*>(q_dev) + q0 * row, static_cast<const uint8_t*>(q_host) + q0 * row, nq * row, hs->in) &&
+         h2d(static_cast<uint8_t*>(k_dev) + k0 * row, static_cast<const uint8_t*>(k_host) + k0 * row, nk * row, hs->in) &&
+         h2d(static_cast<uint8_t*>(v_dev) + k0 * row, static_cast<const uint8_t*>(v_host) + k0 * row, nk * row, hs->in) &&
+         hs->write32(reinterpret_cast<CUstream>(hs->in), fl + 4 * (kPieceReady + c), 1u, 0) == CUDA_SUCCESS;
+  }
+  // (Recorded whatever happened above, so that the join below also covers
+  // copies and ready words queued before a failure.)
+  const bool in_recorded = cudaEventRecord(hs->in_done, hs->in) == cudaSuccess;
+  ok = ok && in_recorded;
+  // The pass, before any copy out is queued: a copy out of pageable memory
+  // returns only when done, and must not wait for a kernel not yet launched.
+  if (ok) st = launch_v2_on<false>(q_dev, k_dev, v_dev, p, s, flags);
+  if (!ok && st == FP8ATTN_OK) st = FP8ATTN_ERR_CUDA;
+  // Copies out: each piece once its flag is up (the kernel raises every flag,
+  // also when it gives up, so these waits always end once it has run).
+  for (int c = 0; st == FP8ATTN_OK && c < n_pieces; ++c) {
+    const size_t q0 = static_cast<size_t>(c) * p.heads_per_piece;
+    const size_t nq = std::min<size_t>(p.heads_per_piece, zq - q0);
+    if (hs->wait32(reinterpret_cast<CUstream>(hs->out), fl + 4 * (kPieceFlag + c), 1u, 0 /* GEQ */) != CUDA_SUCCESS ||
+        !d2h(static_cast<uint8_t*>(o_host) + q0 * row * 2, static_cast<const uint8_t*>(o_dev) + q0 * row * 2,
+             nq * row * 2, hs->out) ||
+        (lse_dev && !d2h(lse_host + q0 * N, lse_dev + q0 * N, nq * N * sizeof(float), hs->out)))
+      st = FP8ATTN_ERR_CUDA;
+  }
+  // Join: the stream continues once the copies out (and in) are done; the
+  // block may be handed out again once the stream is past that point.
+  if (cudaEventRecord(hs->out_done, hs->out) != cudaSuccess || cudaStreamWaitEvent(s, hs->out_done, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(s, hs->in_done, 0) != cudaSuccess || cudaEventRecord(hs->block_free[slot], s) != cudaSuccess)
+    st = FP8ATTN_ERR_CUDA;
+  return st;
+}
 
 using namespace fp8attn;
 

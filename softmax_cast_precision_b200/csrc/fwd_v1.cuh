@@ -49,7 +49,21 @@ struct FwdParams {
   // of the first K tile, so that a wait runs out on purpose.
   unsigned long long wait_limit_ns;
   int test_withhold_k;
+  // Persistent kernel, streamed host calls (nullptr otherwise): the inputs
+  // arrive piece by piece, a piece being heads_per_piece consecutive (b, h)
+  // slabs.  Word kPieceReady + c is set by the copy stream once piece c is on
+  // the device; the kernel counts finished query tiles in kPieceDone + c and
+  // sets kPieceFlag + c when piece c's outputs are all stored.
+  unsigned int* stream_flags;
+  int heads_per_piece;
 };
+
+// Word offsets in FwdParams::stream_flags (word 0 is the work-unit counter
+// when the same block holds both).
+constexpr int kPieceReady = 16;
+constexpr int kPieceDone = 32;
+constexpr int kPieceFlag = 48;
+constexpr int kMaxPieces = 16;
 
 template <int D>
 struct V1Config {

@@ -165,6 +165,47 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Streamed calls: wait until piece c of the inputs is on the device (the
+// copy stream sets its ready word after the piece's copies), then order the
+// tensor-memory loads that follow after the copies.  Bounded like every
+// other wait; on timeout the CTA aborts.
+__device__ __forceinline__ bool wait_piece_ready(const FwdParams& p, int c, V2Bars* bars, uint32_t* err_word) {
+  const unsigned int* w = p.stream_flags + kPieceReady + c;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(w) : "memory");
+    if (v != 0u) break;
+    if (bars->abort) return false;
+    if (globaltimer_ns() - t0 > bars->wait_limit_ns) {
+      atomicOr(err_word, kErrTimeoutLoad);
+      bars->abort = 1u;
+      return false;
+    }
+    __nanosleep(1000);
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
+}
+
+// Streamed calls: each of the four warps of a query tile arrives once on its
+// piece after storing its rows of O and lse; the arrival that completes the
+// piece raises the piece's flag for the copy stream.
+__device__ __forceinline__ void piece_tile_stored(const FwdParams& p, int zq, int lane) {
+  __syncwarp();
+  if (lane == 0) {
+    const int c = zq / p.heads_per_piece;
+    const int heads = min(p.heads_per_piece, p.B * p.H - c * p.heads_per_piece);
+    const unsigned int expected = 4u * static_cast<unsigned int>(heads) * static_cast<unsigned int>(p.num_q_tiles);
+    __threadfence();
+    const unsigned int before = atomicAdd(p.stream_flags + kPieceDone + c, 1u);
+    if (before + 1u == expected) {
+      __threadfence_system();
+      atomicExch(p.stream_flags + kPieceFlag + c, 1u);
+    }
+  }
+}
+
 // Readers of each published unit id: lane 0 of the two MMA warps and every
 // thread of the two softmax warpgroups.
 constexpr uint32_t kUnitReaders = 2 + 256;
@@ -255,6 +296,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       uint32_t kv_it = 0, q_it = 0, q_done[2] = {0, 0};
+      int ready_piece = -1;  // streamed calls: the last piece seen on the device
       bool ok = true;
       for (uint32_t u_it = 0; ok; ++u_it) {
         // Claim the next unit and publish it (slot reuse waits until every
@@ -268,6 +310,10 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         mbar_arrive(&bars->unit_full[slot]);
         if (u < 0) break;
         const UnitGeom g = unit_geom(p, u);
+        if (p.stream_flags != nullptr && g.zq / p.heads_per_piece != ready_piece) {
+          ready_piece = g.zq / p.heads_per_piece;
+          if (!wait_piece_ready(p, ready_piece, bars, err_word)) break;
+        }
         if (q_it > 0) ok = v2_wait(bars, &bars->q_free, (q_it - 1) & 1, err_word, kErrTimeoutPipe);
         if (!ok) break;
         // A Q or K tile is one box, or for bfloat16 two boxes of 64 columns
@@ -711,6 +757,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         if (p.lse != nullptr && row < p.N)
           p.lse[static_cast<int64_t>(g.zq) * p.N + row] =
               ((SCALED ? m : m * p.scale_log2) + (log2f(l) - p.log2_p_scale)) * 0.6931471805599453f;
+        if (p.stream_flags != nullptr) piece_tile_stored(p, g.zq, lane);
       }
       tc_fence_before();
       mbar_arrive(&bars->o_free[k]);
@@ -719,6 +766,12 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (p.stream_flags != nullptr && bars->abort && tid == 0) {
+    // This CTA gave up: raise every piece flag, so that no copy stream waits
+    // for outputs that will not come (the error word reports the failure).
+    const int pieces = (p.B * p.H + p.heads_per_piece - 1) / p.heads_per_piece;
+    for (int c = 0; c < pieces; ++c) atomicExch(p.stream_flags + kPieceFlag + c, 1u);
+  }
   if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);

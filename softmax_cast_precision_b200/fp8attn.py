@@ -52,6 +52,8 @@ def lib() -> ctypes.CDLL:
         L.fp8attn_fwd.restype = i32
         L.fp8attn_fwd_noalloc.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, P]
         L.fp8attn_fwd_noalloc.restype = i32
+        L.fp8attn_fwd_host.argtypes = [P, P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, i32, P]
+        L.fp8attn_fwd_host.restype = i32
         L.fp8attn_quantize.argtypes = [P, i32, P, P, i32, i32, i32, i32, P, P]
         L.fp8attn_quantize.restype = i32
         L.fp8attn_fwd_scaled.argtypes = [P, P, P, P, P, P, P, P, P, i32, i32, i32, i32, i32, i32, f32, i32, P]
@@ -173,98 +175,50 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_sc
     return o, lse
 
 
-def host_chunks(B: int, H: int, Hkv: int, N: int, chunks: int | None = None) -> list[tuple[int, int, int]]:
-    """The pieces ``fwd_host`` cuts a problem into: (b, kv head start, kv head end) triples, each within one
-    batch entry, covering every (batch, kv head) once, in order.  ``chunks`` is the target count (default:
-    about eight, fewer when a piece would hold under two waves of 148 persistent CTAs' work units); each
-    batch entry's kv heads are split into near-equal contiguous ranges."""
-    if B <= 0 or Hkv <= 0 or H % Hkv:
-        raise ValueError("need B >= 1, Hkv >= 1 and H a multiple of Hkv")
-    if chunks is None:
-        units = B * H * max(1, -(-N // 256))
-        chunks = max(1, min(8, units // (2 * 148)))
-    per_batch = max(1, min(Hkv, -(-int(chunks) // B)))
-    base, extra = divmod(Hkv, per_batch)
-    out = []
-    for b in range(B):
-        g0 = 0
-        for i in range(per_batch):
-            g1 = g0 + base + (1 if i < extra else 0)
-            out.append((b, g0, g1))
-            g0 = g1
-    return out
-
-
 def fwd_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, causal: bool, p_scale: float = 256.0,
-             kv_order="reverse", chunks: int | None = None, device=None, out: torch.Tensor | None = None,
-             lse_out: torch.Tensor | None = None):
-    """Forward pass of host tensors with the host<->device copies overlapped with the computation.
+             kv_order="reverse", pieces: int = 0, with_lse: bool = True, device=None, out: torch.Tensor | None = None,
+             lse_out: torch.Tensor | None = None, stream=None):
+    """Forward pass of host tensors, the copies overlapped with the computation (C entry ``fp8attn_fwd_host``).
 
-    q [B,H,N,d], k, v [B,Hkv,N,d] are E4M3 host tensors (pinned, for the copies to overlap).  The problem is
-    cut into pieces of whole kv heads with their query heads (``host_chunks``); piece c is copied to the device
-    on one stream, computed by ``fp8attn_fwd`` once its copy is done, and copied back on a third stream, so that
-    the copies of one piece run during the computation of the others.  The pieces' passes alternate between two
-    streams, so that one piece's persistent kernel can start on the SMs the previous one has finished with.
-    Returns host (o, lse): ``out`` (bfloat16 [B,H,N,d]) and ``lse_out`` (float32 [B,H,N]) when given (pinned,
-    for the copies to overlap), else new pinned tensors.  The call returns once both are complete.
+    q [B,H,N,d], k, v [B,Hkv,N,d] are E4M3 host tensors (pinned, for the copies to overlap).  The library cuts
+    the problem into ``pieces`` pieces of whole kv heads (0: its default), copies each in on a copy stream of its
+    own, runs one persistent pass on ``stream`` (default: the device's current stream) that takes the pieces in
+    order as they land, and copies each piece's outputs back as soon as they are stored.  Device staging buffers
+    are allocated here.  Returns host (o, lse): ``out`` (bfloat16 [B,H,N,d]) and ``lse_out`` (float32 [B,H,N])
+    when given (pinned, for the copies to overlap), else new pinned tensors; lse is None when ``with_lse`` is
+    False.  The call returns once both are complete.
     """
     q, k, v = _bytes(q), _bytes(k), _bytes(v)
     B, H, Hkv, N, d = _shapes(q, k, v)
     if q.is_cuda or k.is_cuda or v.is_cuda:
         raise ValueError("fwd_host takes host tensors")
+    if not all(t.is_contiguous() for t in (q, k, v)):
+        raise ValueError("fwd_host takes contiguous q, k, v")
     dev = torch.device(device if device is not None else "cuda:0")
-    rep = H // Hkv
-    o_h = out if out is not None else torch.empty((B, H, N, d), dtype=torch.bfloat16, pin_memory=True)
-    lse_h = lse_out if lse_out is not None else torch.empty((B, H, N), dtype=torch.float32, pin_memory=True)
-    if (o_h.is_cuda or lse_h.is_cuda or o_h.dtype != torch.bfloat16 or lse_h.dtype != torch.float32
-            or tuple(o_h.shape) != (B, H, N, d) or tuple(lse_h.shape) != (B, H, N)
-            or not o_h.is_contiguous() or not lse_h.is_contiguous()):
+    if ((out is not None and (out.is_cuda or out.dtype != torch.bfloat16 or tuple(out.shape) != (B, H, N, d)
+                              or not out.is_contiguous()))
+            or (with_lse and lse_out is not None and (lse_out.is_cuda or lse_out.dtype != torch.float32
+                                                      or tuple(lse_out.shape) != (B, H, N)
+                                                      or not lse_out.is_contiguous()))):
         raise ValueError("out / lse_out must be contiguous host tensors: bfloat16 [B,H,N,d] and float32 [B,H,N]")
+    o_h = out if out is not None else torch.empty((B, H, N, d), dtype=torch.bfloat16, pin_memory=True)
+    lse_h = None
+    if with_lse:
+        lse_h = lse_out if lse_out is not None else torch.empty((B, H, N), dtype=torch.float32, pin_memory=True)
     if B * H * N == 0:
         return o_h, lse_h
     qd, kd, vd = (torch.empty(t.shape, dtype=torch.uint8, device=dev) for t in (q, k, v))
     od = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=dev)
-    lsed = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-    main = torch.cuda.current_stream(dev)
-    s_in, s_c0, s_c1, s_out = (torch.cuda.Stream(device=dev) for _ in range(4))
-    for s in (s_in, s_c0, s_c1, s_out):
-        s.wait_stream(main)  # the buffers above were allocated on the current stream
-    L = lib()
-    done = torch.cuda.Event()
+    lsed = torch.empty((B, H, N), dtype=torch.float32, device=dev) if lse_h is not None else None
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
     with _on_device(dev):
-        _fwd_host_pieces(L, q, k, v, qd, kd, vd, od, lsed, o_h, lse_h, B, H, Hkv, N, d, rep, causal, p_scale,
-                         kv_order, chunks, dev, s_in, s_c0, s_c1, s_out)
-    done.record(s_out)
-    main.wait_event(done)  # work ordered after this call on the current stream follows the copies out
-    done.synchronize()
+        st = lib().fp8attn_fwd_host(_ptr(q), _ptr(k), _ptr(v), _ptr(o_h), _ptr(lse_h), _ptr(qd), _ptr(kd), _ptr(vd),
+                                    _ptr(od), _ptr(lsed), B, H, Hkv, N, d, int(bool(causal)), ctypes.c_float(p_scale),
+                                    _order(kv_order), int(pieces), ctypes.c_void_p(s.cuda_stream))
+    if st != OK:
+        raise Fp8AttnError(st, "fp8attn_fwd_host")
+    s.synchronize()
     return o_h, lse_h
-
-
-def _fwd_host_pieces(L, q, k, v, qd, kd, vd, od, lsed, o_h, lse_h, B, H, Hkv, N, d, rep, causal, p_scale, kv_order,
-                     chunks, dev, s_in, s_c0, s_c1, s_out):
-    """The piece loop of ``fwd_host``: copy in, compute (alternating s_c0 / s_c1), copy out."""
-    for c, (b, g0, g1) in enumerate(host_chunks(B, H, Hkv, N, chunks)):
-        s_comp = s_c1 if c & 1 else s_c0
-        h0, h1 = g0 * rep, g1 * rep
-        with torch.cuda.stream(s_in):
-            qd[b, h0:h1].copy_(q[b, h0:h1], non_blocking=True)
-            kd[b, g0:g1].copy_(k[b, g0:g1], non_blocking=True)
-            vd[b, g0:g1].copy_(v[b, g0:g1], non_blocking=True)
-        landed = torch.cuda.Event()
-        landed.record(s_in)
-        s_comp.wait_event(landed)
-        st = L.fp8attn_fwd(_ptr(qd[b, h0:h1]), _ptr(kd[b, g0:g1]), _ptr(vd[b, g0:g1]), _ptr(od[b, h0:h1]),
-                           _ptr(lsed[b, h0:h1]), 1, h1 - h0, g1 - g0, N, d, int(bool(causal)), ctypes.c_float(p_scale),
-                           _order(kv_order), ctypes.c_void_p(s_comp.cuda_stream))
-        if st != OK:
-            torch.cuda.synchronize(dev)
-            raise Fp8AttnError(st, "fp8attn_fwd")
-        computed = torch.cuda.Event()
-        computed.record(s_comp)
-        s_out.wait_event(computed)
-        with torch.cuda.stream(s_out):
-            o_h[b, h0:h1].copy_(od[b, h0:h1], non_blocking=True)
-            lse_h[b, h0:h1].copy_(lsed[b, h0:h1], non_blocking=True)
 
 
 def fwd_noalloc(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, out: torch.Tensor,
