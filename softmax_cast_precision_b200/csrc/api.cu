@@ -171,7 +171,9 @@ int launch_v2_on(const void* q, const void* k, const void* v, FwdParams p, cudaS
                             : (make_map(&tq, q, 128, p.N, p.B * p.H, 128) &&
                                make_map(&tk, k, 128, p.N, p.B * p.Hkv, 128));
   if (!maps_ok || !make_map(&tv, v, 128, p.N, p.B * p.Hkv, 128)) return FP8ATTN_ERR_CUDA;
-  auto kern = fwd_v2_kernel<COUNT, SCALED, QK16>;
+  // Streamed calls take their own instance (plain forward pass only).
+  if (p.stream_flags != nullptr && (COUNT || SCALED || QK16)) return FP8ATTN_ERR_UNSUPPORTED;
+  auto kern = p.stream_flags != nullptr ? fwd_v2_kernel<false, false, false, true> : fwd_v2_kernel<COUNT, SCALED, QK16>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess)
     return FP8ATTN_ERR_CUDA;
   // The warpgroups re-split the block's registers with setmaxnreg; that split
@@ -759,8 +761,8 @@ extern "C" int fp8attn_bwd(const void* q, const void* k, const void* v, const vo
     return FP8ATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   bwd_delta_kernel<<<static_cast<unsigned int>((rows + 7) / 8), 256, 0, s>>>(p);
-  bwd_dkdv_kernel<<<dim3(p.num_tiles, Hkv, B), 128, DkdvLayout::SMEM_BYTES, s>>>(tq, tk, tv, tdo, p, err_word);
-  bwd_dq_kernel<<<dim3(p.num_tiles, H, B), 128, DqLayout::SMEM_BYTES, s>>>(tq, tk, tv, tdo, p, err_word);
+  bwd_dkdv_kernel<<<dim3(p.num_tiles, Hkv, B), 256, DkdvLayout::SMEM_BYTES, s>>>(tq, tk, tv, tdo, p, err_word);
+  bwd_dq_kernel<<<dim3(p.num_tiles, H, B), 256, DqLayout::SMEM_BYTES, s>>>(tq, tk, tv, tdo, p, err_word);
   return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
 }
 

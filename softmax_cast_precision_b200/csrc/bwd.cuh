@@ -74,12 +74,11 @@ struct BwdConfig {
 // Shared-memory layout of bwd_dkdv_kernel (offsets from a 1024-byte aligned base).
 struct DkdvLayout {
   static constexpr int OFF_K = 0;                                   // K_j   E4M3
-  static constexpr int OFF_VF = OFF_K + BwdConfig::F8_TILE;         // V_j   E4M3 (converted once)
-  static constexpr int OFF_VB = OFF_VF + BwdConfig::F8_TILE;        // V_j   bf16
-  static constexpr int OFF_Q = OFF_VB + BwdConfig::BF_TILE;         // Q_i   E4M3
+  static constexpr int OFF_VB = OFF_K + BwdConfig::F8_TILE;         // V_j   bf16
+  static constexpr int OFF_Q = OFF_VB + BwdConfig::BF_TILE;         // Q_i   E4M3 (first V_j E4M3, converted once)
   static constexpr int OFF_QB = OFF_Q + BwdConfig::F8_TILE;         // Q_i   bf16
-  static constexpr int OFF_DO = OFF_QB + BwdConfig::BF_TILE;        // dO_i  bf16
-  static constexpr int OFF_PT = OFF_DO + BwdConfig::BF_TILE;        // E4M3(P^T S) as bf16
+  static constexpr int OFF_DO = OFF_QB + BwdConfig::BF_TILE;        // dO_i  bf16, two buffers (step parity)
+  static constexpr int OFF_PT = OFF_DO + 2 * BwdConfig::BF_TILE;    // E4M3(P^T S) as bf16
   static constexpr int OFF_DST = OFF_PT + BwdConfig::BF_TILE;       // dS^T  bf16
   static constexpr int OFF_VEC = OFF_DST + BwdConfig::BF_TILE;      // lse_i * log2(e) [128], D_i [128]
   static constexpr int OFF_BAR = OFF_VEC + 2 * 128 * 4;
@@ -92,8 +91,8 @@ struct DqLayout {
   static constexpr int OFF_DO = OFF_Q + BwdConfig::F8_TILE;         // dO_i  bf16
   static constexpr int OFF_K = OFF_DO + BwdConfig::BF_TILE;         // K_j   E4M3
   static constexpr int OFF_V = OFF_K + BwdConfig::F8_TILE;          // V_j   E4M3
-  static constexpr int OFF_KB = OFF_V + BwdConfig::F8_TILE;         // K_j   bf16
-  static constexpr int OFF_VB = OFF_KB + BwdConfig::BF_TILE;        // V_j   bf16
+  static constexpr int OFF_KB = OFF_V + BwdConfig::F8_TILE;         // K_j   bf16, two buffers (step parity)
+  static constexpr int OFF_VB = OFF_KB + 2 * BwdConfig::BF_TILE;    // V_j   bf16
   static constexpr int OFF_DS = OFF_VB + BwdConfig::BF_TILE;        // dS    bf16
   static constexpr int OFF_BAR = OFF_DS + BwdConfig::BF_TILE;
   static constexpr int SMEM_BYTES = OFF_BAR + 128 + 1024;
@@ -102,7 +101,7 @@ struct DqLayout {
 // Every swizzled tile starts on a 1024-byte boundary (the 128-byte swizzle
 // pattern repeats every 8 rows of 128 bytes and is keyed to address bits
 // 7..9), and each kernel fits the 227 KB a CTA may opt into.
-static_assert(DkdvLayout::OFF_VF % 1024 == 0 && DkdvLayout::OFF_VB % 1024 == 0 && DkdvLayout::OFF_Q % 1024 == 0 &&
+static_assert(DkdvLayout::OFF_VB % 1024 == 0 && DkdvLayout::OFF_Q % 1024 == 0 &&
                   DkdvLayout::OFF_QB % 1024 == 0 && DkdvLayout::OFF_DO % 1024 == 0 &&
                   DkdvLayout::OFF_PT % 1024 == 0 && DkdvLayout::OFF_DST % 1024 == 0,
               "dK/dV tiles must be 1024-byte aligned");
@@ -152,6 +151,29 @@ __device__ __forceinline__ void bwd_convert_row(const uint8_t* src, uint8_t* dst
                  : "r"(s + r * 128 + ((c ^ (r & 7)) << 4))
                  : "memory");
     // 16 E4M3 columns 16c .. 16c+15 become bfloat16 chunks 2c and 2c+1.
+    const uint2 a = bwd_e4m3x4_to_bf16x4(w0), b = bwd_e4m3x4_to_bf16x4(w1);
+    const uint2 e = bwd_e4m3x4_to_bf16x4(w2), f = bwd_e4m3x4_to_bf16x4(w3);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d + bf16_tile_chunk(r, 2 * c)), "r"(a.x),
+                 "r"(a.y), "r"(b.x), "r"(b.y)
+                 : "memory");
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d + bf16_tile_chunk(r, 2 * c + 1)), "r"(e.x),
+                 "r"(e.y), "r"(f.x), "r"(f.y)
+                 : "memory");
+  }
+}
+
+// Half of that: E4M3 columns 64 h .. 64 h + 63 of row `r` (h = 0, 1), so
+// that two threads share the conversion of a row.
+__device__ __forceinline__ void bwd_convert_half_row(const uint8_t* src, uint8_t* dst, int r, int h) {
+  const uint32_t s = smem_u32(src), d = smem_u32(dst);
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const int c = 4 * h + cc;
+    uint32_t w0, w1, w2, w3;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
+                 : "r"(s + r * 128 + ((c ^ (r & 7)) << 4))
+                 : "memory");
     const uint2 a = bwd_e4m3x4_to_bf16x4(w0), b = bwd_e4m3x4_to_bf16x4(w1);
     const uint2 e = bwd_e4m3x4_to_bf16x4(w2), f = bwd_e4m3x4_to_bf16x4(w3);
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d + bf16_tile_chunk(r, 2 * c)), "r"(a.x),
@@ -227,7 +249,7 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const BwdParams p) {
 // --------------------------------------------------------------------------
 // dK and dV: one CTA (one warpgroup) per (batch, kv head, key tile).
 // --------------------------------------------------------------------------
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const BwdParams p, uint32_t* err_word) {
@@ -237,13 +259,17 @@ __global__ void __launch_bounds__(128, 1)
   float* sLse2 = reinterpret_cast<float*>(base + L::OFF_VEC);
   float* sDelta = sLse2 + 128;
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
-  uint64_t* bar_kv = bars + 0;  // K_j and V_j landed
-  uint64_t* bar_q = bars + 1;   // Q_i and dO_i landed
-  uint64_t* bar_s = bars + 2;   // S^T and dP^T computed
-  uint64_t* bar_g = bars + 3;   // dV and dK products of this step complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  uint64_t* bar_kv = bars + 0;     // K_j and V_j landed
+  uint64_t* bar_q = bars + 1;      // Q_i landed
+  uint64_t* bar_do = bars + 2;     // dO_i landed, one barrier per buffer (step parity)
+  uint64_t* bar_s = bars + 4;      // S^T and dP^T computed
+  uint64_t* bar_g = bars + 5;      // dV and dK products of this step complete
+  uint64_t* bar_drain = bars + 6;  // every product issued so far complete (abort path)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  // Two warpgroups: thread tid owns TMEM lane (key row) r = tid % 128 and, in
+  // each step, half wg = tid / 128 of the queries: chunks 2 wg and 2 wg + 1.
+  const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, r = tid & 127;
   const int jt = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int k0 = jt * 128;
   const int zkv = b * p.Hkv + hk;
@@ -252,7 +278,7 @@ __global__ void __launch_bounds__(128, 1)
   const int n_iter = p.h_per_kv * per_head;
 
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < 7; ++i) mbar_init(bars + i, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -268,52 +294,85 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
 
   auto step_geom = [&](int it, int& zq, int& q0) {
     const int hl = it / per_head;
     q0 = (i_first + (it - hl * per_head)) * 128;
     zq = b * p.H + hk * p.h_per_kv + hl;
   };
+  // Thread 0's loads.  Q_i has one buffer: step it + 1's is fetched once
+  // S^T(it) is complete (Q(it) is already converted by then).  dO has two:
+  // step it + 2's goes to step it's buffer once step it's products are
+  // complete.  Issued / waited counts drive the drain after an abort.
+  int q_issued = 0, q_landed = 0, do_issued = 0, do_landed = 0;
   auto issue_q = [&](int it) {
     int zq, q0;
     step_geom(it, zq, q0);
-    mbar_arrive_expect_tx(bar_q, BwdConfig::F8_TILE + BwdConfig::BF_TILE);
+    ++q_issued;
+    mbar_arrive_expect_tx(bar_q, BwdConfig::F8_TILE);
     tma_load_3d(base + L::OFF_Q, &tm_q, bar_q, 0, q0, zq);
-    tma_load_3d(base + L::OFF_DO, &tm_do, bar_q, 0, q0, zq);
-    tma_load_3d(base + L::OFF_DO + BwdConfig::BF_PANEL, &tm_do, bar_q, 64, q0, zq);
+  };
+  auto issue_do = [&](int it) {
+    int zq, q0;
+    step_geom(it, zq, q0);
+    ++do_issued;
+    uint8_t* dst = base + L::OFF_DO + (it & 1) * BwdConfig::BF_TILE;
+    mbar_arrive_expect_tx(bar_do + (it & 1), BwdConfig::BF_TILE);
+    tma_load_3d(dst, &tm_do, bar_do + (it & 1), 0, q0, zq);
+    tma_load_3d(dst + BwdConfig::BF_PANEL, &tm_do, bar_do + (it & 1), 64, q0, zq);
   };
   if (tid == 0) {
+    // V_j (E4M3) lands in the Q buffer, to be converted once.
     mbar_arrive_expect_tx(bar_kv, 2 * BwdConfig::F8_TILE);
     tma_load_3d(base + L::OFF_K, &tm_k, bar_kv, 0, k0, zkv);
-    tma_load_3d(base + L::OFF_VF, &tm_v, bar_kv, 0, k0, zkv);
-    issue_q(0);
+    tma_load_3d(base + L::OFF_Q, &tm_v, bar_kv, 0, k0, zkv);
+    if (n_iter > 0) issue_do(0);
+    if (n_iter > 1) issue_do(1);
   }
 
   const uint32_t sK = smem_u32(base + L::OFF_K), sVB = smem_u32(base + L::OFF_VB);
   const uint32_t sQ = smem_u32(base + L::OFF_Q), sQB = smem_u32(base + L::OFF_QB);
-  const uint32_t sDO = smem_u32(base + L::OFF_DO), sPT = smem_u32(base + L::OFF_PT);
-  const uint32_t sDST = smem_u32(base + L::OFF_DST);
+  const uint32_t sPT = smem_u32(base + L::OFF_PT), sDST = smem_u32(base + L::OFF_DST);
   constexpr uint32_t idesc_s = idesc_e4m3_f32(128, 128, false, false);      // S^T = K Q^T
   constexpr uint32_t idesc_dp = bwd_idesc_bf16(128, 128, false, false);     // dP^T = V dO^T
   constexpr uint32_t idesc_grad = bwd_idesc_bf16(128, 128, false, true);    // dV += P^T dO, dK += dS^T Q
 
-  const int key = k0 + tid;  // this thread's TMEM lane: one key
+  const int key = k0 + r;  // this thread's TMEM lane: one key
   bool fail = !mbar_wait_bounded(bar_kv, 0, err_word, kErrTimeoutKV);
-  if (!fail) bwd_convert_row(base + L::OFF_VF, base + L::OFF_VB, tid);
-  bool abort = false;
+  if (!fail) bwd_convert_half_row(base + L::OFF_Q, base + L::OFF_VB, r, wg);
+  // Every thread has read V out of the Q buffer before Q_0 may overwrite it.
+  fence_proxy_async_smem();
+  bool abort = __syncthreads_or(fail) != 0;
+  if (!abort && tid == 0 && n_iter > 0) issue_q(0);
+  // lse (warpgroup 0) and D (warpgroup 1) of the step's 128 queries, fetched
+  // one step ahead.
+  auto fetch_vec = [&](int it) -> float {
+    float x = 0.0f;
+    if (it < n_iter) {
+      int zq, q0;
+      step_geom(it, zq, q0);
+      const int qi = q0 + r;
+      if (qi < p.N) {
+        const int64_t idx = static_cast<int64_t>(zq) * p.N + qi;
+        x = wg == 0 ? p.lse[idx] * 1.4426950408889634f : p.delta[idx];
+      }
+    }
+    return x;
+  };
+  float next_vec = fetch_vec(0);
 
-  for (int it = 0; it < n_iter; ++it) {
+  for (int it = 0; !abort && it < n_iter; ++it) {
+    (wg == 0 ? sLse2 : sDelta)[r] = next_vec;
+    next_vec = fetch_vec(it + 1);
+    const uint32_t sDO = smem_u32(base + L::OFF_DO + (it & 1) * BwdConfig::BF_TILE);
     int zq, q0;
     step_geom(it, zq, q0);
-    {
-      const int qi = q0 + tid;
-      const int64_t idx = static_cast<int64_t>(zq) * p.N + qi;
-      sLse2[tid] = qi < p.N ? p.lse[idx] * 1.4426950408889634f : 0.0f;
-      sDelta[tid] = qi < p.N ? p.delta[idx] : 0.0f;
-    }
     if (!fail && !mbar_wait_bounded(bar_q, it & 1, err_word, kErrTimeoutQ)) fail = true;
-    if (!fail) bwd_convert_row(base + L::OFF_Q, base + L::OFF_QB, tid);
+    if (!fail && tid == 0) q_landed = it + 1;
+    if (!fail && !mbar_wait_bounded(bar_do + (it & 1), (it >> 1) & 1, err_word, kErrTimeoutQ)) fail = true;
+    if (!fail && tid == 0) do_landed = it + 1;
+    if (!fail) bwd_convert_half_row(base + L::OFF_Q, base + L::OFF_QB, r, wg);
     fence_proxy_async_smem();
     tc_fence_before();
     abort = __syncthreads_or(fail) != 0;
@@ -332,10 +391,13 @@ __global__ void __launch_bounds__(128, 1)
     }
     if (!mbar_wait_bounded(bar_s, it & 1, err_word, kErrTimeoutMMA)) fail = true;
     tc_fence_after();
+    // S^T(it) has read Q(it), which is converted already: fetch the next Q.
+    if (tid == 0 && !fail && it + 1 < n_iter) issue_q(it + 1);
 
-    // P^T, E4M3(P^T S) and dS^T for this thread's key, 32 queries at a time.
+    // P^T, E4M3(P^T S) and dS^T for this thread's key and half of the
+    // queries, 32 at a time.
 #pragma unroll 1
-    for (int g = 0; g < 4; ++g) {
+    for (int g = 2 * wg; g < 2 * wg + 2; ++g) {
       uint32_t rs[32], rdp[32];
       tmem_ld32(tS + lane_off + 32 * g, rs);
       tmem_ld32(tDP + lane_off + 32 * g, rdp);
@@ -350,8 +412,8 @@ __global__ void __launch_bounds__(128, 1)
         ph[e] = bwd_e4m3_value(pr * p.p_scale);
         ds[e] = pr * (__uint_as_float(rdp[e]) - sDelta[c]);
       }
-      bwd_store_bf16_32(base + L::OFF_PT, tid, g, ph);
-      bwd_store_bf16_32(base + L::OFF_DST, tid, g, ds);
+      bwd_store_bf16_32(base + L::OFF_PT, r, g, ph);
+      bwd_store_bf16_32(base + L::OFF_DST, r, g, ds);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -372,34 +434,44 @@ __global__ void __launch_bounds__(128, 1)
     }
     if (!mbar_wait_bounded(bar_g, it & 1, err_word, kErrTimeoutMMA)) fail = true;
     tc_fence_after();
-    // Q, dO and the converted tiles are free again: fetch the next step's.
-    if (tid == 0 && !fail && it + 1 < n_iter) issue_q(it + 1);
+    // This step's dO buffer is free again: fetch the dO of the step after next.
+    if (tid == 0 && !fail && it + 2 < n_iter) issue_do(it + 2);
   }
   abort = __syncthreads_or(fail || abort) != 0;
 
   if (!abort) {
-    // Every lane takes part in the warp-wide TMEM loads; lanes past N store nothing.
+    // Warpgroup 0 writes dV / S, warpgroup 1 dK / sqrt(d).  Every lane takes
+    // part in the warp-wide TMEM loads; lanes past N store nothing.
     const int64_t row = static_cast<int64_t>(zkv) * p.N + key;
-    float* dvrow = p.dv + row * 128;
-    float* dkrow = p.dk + row * 128;
+    float* dst = (wg == 0 ? p.dv : p.dk) + row * 128;
 #pragma unroll 1
     for (int g = 0; g < 4; ++g) {
-      uint32_t a[32], c[32];
-      tmem_ld32(tDV + lane_off + 32 * g, a);
-      tmem_ld32(tDK + lane_off + 32 * g, c);
+      uint32_t a[32];
+      tmem_ld32((wg == 0 ? tDV : tDK) + lane_off + 32 * g, a);
       tmem_wait_ld();
       if (key < p.N) {
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          reinterpret_cast<float4*>(dvrow + 32 * g)[e / 4] = make_float4(
-              __fdiv_rn(__uint_as_float(a[e]), p.p_scale), __fdiv_rn(__uint_as_float(a[e + 1]), p.p_scale),
-              __fdiv_rn(__uint_as_float(a[e + 2]), p.p_scale), __fdiv_rn(__uint_as_float(a[e + 3]), p.p_scale));
-          reinterpret_cast<float4*>(dkrow + 32 * g)[e / 4] =
-              make_float4(__uint_as_float(c[e]) * p.inv_sqrt_d, __uint_as_float(c[e + 1]) * p.inv_sqrt_d,
-                          __uint_as_float(c[e + 2]) * p.inv_sqrt_d, __uint_as_float(c[e + 3]) * p.inv_sqrt_d);
+          float4 x;
+          if (wg == 0)
+            x = make_float4(__fdiv_rn(__uint_as_float(a[e]), p.p_scale), __fdiv_rn(__uint_as_float(a[e + 1]), p.p_scale),
+                            __fdiv_rn(__uint_as_float(a[e + 2]), p.p_scale), __fdiv_rn(__uint_as_float(a[e + 3]), p.p_scale));
+          else
+            x = make_float4(__uint_as_float(a[e]) * p.inv_sqrt_d, __uint_as_float(a[e + 1]) * p.inv_sqrt_d,
+                            __uint_as_float(a[e + 2]) * p.inv_sqrt_d, __uint_as_float(a[e + 3]) * p.inv_sqrt_d);
+          reinterpret_cast<float4*>(dst + 32 * g)[e / 4] = x;
         }
       }
     }
+  } else if (tid == 0) {
+    // A wait ran out: let the products and loads still in flight land before
+    // the CTA's tensor and shared memory are released (each wait again bounded).
+    mma_commit(bar_drain);
+    mbar_wait_bounded(bar_drain, 0, err_word, kErrTimeoutMMA, 100000000ull);
+    mbar_wait_bounded(bar_kv, 0, err_word, kErrTimeoutKV, 100000000ull);
+    for (int j = q_landed; j < q_issued; ++j) mbar_wait_bounded(bar_q, j & 1, err_word, kErrTimeoutQ, 100000000ull);
+    for (int j = do_landed; j < do_issued; ++j)
+      mbar_wait_bounded(bar_do + (j & 1), (j >> 1) & 1, err_word, kErrTimeoutQ, 100000000ull);
   }
 
   tc_fence_before();
@@ -413,7 +485,7 @@ __global__ void __launch_bounds__(128, 1)
 // --------------------------------------------------------------------------
 // dQ: one CTA (one warpgroup) per (batch, head, query tile).
 // --------------------------------------------------------------------------
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(256, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const BwdParams p, uint32_t* err_word) {
@@ -424,10 +496,13 @@ __global__ void __launch_bounds__(128, 1)
   uint64_t* bar_q = bars + 0;   // Q_i and dO_i landed
   uint64_t* bar_kv = bars + 1;  // K_j and V_j landed
   uint64_t* bar_s = bars + 2;   // S and dP computed
-  uint64_t* bar_g = bars + 3;   // dQ product of this step complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 4);
+  uint64_t* bar_g = bars + 3;      // dQ product of this step complete
+  uint64_t* bar_drain = bars + 4;  // every product issued so far complete (abort path)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  // Two warpgroups: thread tid owns TMEM lane (query row) r = tid % 128 and,
+  // in each step, half wg = tid / 128 of the keys: chunks 2 wg and 2 wg + 1.
+  const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, r = tid & 127;
   const int it_q = p.num_tiles - 1 - static_cast<int>(blockIdx.x);  // longest causal rows first
   const int h = blockIdx.y, b = blockIdx.z;
   const int q0 = it_q * 128;
@@ -436,7 +511,7 @@ __global__ void __launch_bounds__(128, 1)
   const int last = p.causal ? it_q : p.num_tiles - 1;  // key tiles 0 .. last
 
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < 5; ++i) mbar_init(bars + i, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -452,9 +527,11 @@ __global__ void __launch_bounds__(128, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 256;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
 
+  int kv_issued = 0, kv_landed = 0;  // thread 0: key tiles issued / waited for (drain after an abort)
   auto issue_kv = [&](int j) {
+    kv_issued = j + 1;
     mbar_arrive_expect_tx(bar_kv, 2 * BwdConfig::F8_TILE);
     tma_load_3d(base + L::OFF_K, &tm_k, bar_kv, 0, j * 128, zkv);
     tma_load_3d(base + L::OFF_V, &tm_v, bar_kv, 0, j * 128, zkv);
@@ -474,7 +551,7 @@ __global__ void __launch_bounds__(128, 1)
   constexpr uint32_t idesc_dp = bwd_idesc_bf16(128, 128, false, false);  // dP = dO V^T
   constexpr uint32_t idesc_dq = bwd_idesc_bf16(128, 128, false, true);   // dQ += dS K
 
-  const int row = q0 + tid;  // this thread's TMEM lane: one query
+  const int row = q0 + r;  // this thread's TMEM lane: one query
   const int64_t ridx = static_cast<int64_t>(zq) * p.N + row;
   const float lse2 = row < p.N ? p.lse[ridx] * 1.4426950408889634f : 0.0f;
   const float dlt = row < p.N ? p.delta[ridx] : 0.0f;
@@ -484,9 +561,13 @@ __global__ void __launch_bounds__(128, 1)
   for (int j = 0; j <= last; ++j) {
     const int j0 = j * 128;
     if (!fail && !mbar_wait_bounded(bar_kv, j & 1, err_word, kErrTimeoutKV)) fail = true;
+    if (!fail && tid == 0) kv_landed = j + 1;
     if (!fail) {
-      bwd_convert_row(base + L::OFF_K, base + L::OFF_KB, tid);
-      bwd_convert_row(base + L::OFF_V, base + L::OFF_VB, tid);
+      // Warpgroup 0 converts K, warpgroup 1 V.
+      if (wg == 0)
+        bwd_convert_row(base + L::OFF_K, base + L::OFF_KB + (j & 1) * BwdConfig::BF_TILE, r);
+      else
+        bwd_convert_row(base + L::OFF_V, base + L::OFF_VB, r);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -510,8 +591,10 @@ __global__ void __launch_bounds__(128, 1)
     // the barrier): fetch the next key tile while this one is finished.
     if (tid == 0 && !fail && j < last) issue_kv(j + 1);
 
+    // dS is single-buffered: the previous step's dQ product must have read it.
+    if (j > 0 && !mbar_wait_bounded(bar_g, (j - 1) & 1, err_word, kErrTimeoutMMA)) fail = true;
 #pragma unroll 1
-    for (int g = 0; g < 4; ++g) {
+    for (int g = 2 * wg; g < 2 * wg + 2; ++g) {
       uint32_t rs[32], rdp[32];
       tmem_ld32(tS + lane_off + 32 * g, rs);
       tmem_ld32(tDP + lane_off + 32 * g, rdp);
@@ -524,7 +607,7 @@ __global__ void __launch_bounds__(128, 1)
         const float pr = visible ? ex2_approx(__uint_as_float(rs[e]) * p.scale_log2 - lse2) : 0.0f;
         ds[e] = pr * (__uint_as_float(rdp[e]) - dlt);
       }
-      bwd_store_bf16_32(base + L::OFF_DS, tid, g, ds);
+      bwd_store_bf16_32(base + L::OFF_DS, r, g, ds);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -535,20 +618,23 @@ __global__ void __launch_bounds__(128, 1)
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_bf16_ss(tDQ, kmajor_desc(sDS) + bf16_kmajor_step(kk), bf16_mnmajor_desc(sKB) + 128 * kk, idesc_dq,
-                    (j > 0) || (kk > 0));
+        mma_bf16_ss(tDQ, kmajor_desc(sDS) + bf16_kmajor_step(kk),
+                    bf16_mnmajor_desc(sKB + (j & 1) * BwdConfig::BF_TILE) + 128 * kk, idesc_dq, (j > 0) || (kk > 0));
       mma_commit(bar_g);
     }
-    // The next step rewrites the converted tiles and dS: wait for this product.
-    if (!mbar_wait_bounded(bar_g, j & 1, err_word, kErrTimeoutMMA)) fail = true;
-    tc_fence_after();
+    // Not waited here: the next step converts into the other K buffer and
+    // issues its S and dP behind this product; it waits for this product only
+    // before it rewrites dS.
   }
+  // The last dQ product.
+  if (!abort && last >= 0 && !mbar_wait_bounded(bar_g, last & 1, err_word, kErrTimeoutMMA)) fail = true;
+  tc_fence_after();
   abort = __syncthreads_or(fail || abort) != 0;
 
   if (!abort) {
     float* dqrow = p.dq + ridx * 128;
 #pragma unroll 1
-    for (int g = 0; g < 4; ++g) {
+    for (int g = 2 * wg; g < 2 * wg + 2; ++g) {
       uint32_t a[32];
       tmem_ld32(tDQ + lane_off + 32 * g, a);
       tmem_wait_ld();
@@ -562,6 +648,14 @@ __global__ void __launch_bounds__(128, 1)
     }
   }
 
+  if (abort && tid == 0) {
+    // A wait ran out: let the products and loads still in flight land before
+    // the CTA's tensor and shared memory are released (each wait again bounded).
+    mma_commit(bar_drain);
+    mbar_wait_bounded(bar_drain, 0, err_word, kErrTimeoutMMA, 100000000ull);
+    mbar_wait_bounded(bar_q, 0, err_word, kErrTimeoutQ, 100000000ull);
+    for (int j = kv_landed; j < kv_issued; ++j) mbar_wait_bounded(bar_kv, j & 1, err_word, kErrTimeoutKV, 100000000ull);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

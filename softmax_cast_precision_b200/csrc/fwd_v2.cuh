@@ -224,7 +224,9 @@ constexpr int kPolyPairs = 0;
 // log2 units of the descaled logits, whose scale changes from tile to tile.
 // QK16: Q and K are bfloat16 and S = Q K^T runs as a kind::f16 product (the
 // P-cast and P V are unchanged).
-template <bool COUNT, bool SCALED = false, bool QK16 = false>
+// STREAMED: the inputs arrive piece by piece (FwdParams::stream_flags); its
+// own instance, so that the other instances carry no streaming code.
+template <bool COUNT, bool SCALED = false, bool QK16 = false, bool STREAMED = false>
 __global__ void __launch_bounds__(V2Config::THREADS, 1)
     fwd_v2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p, uint32_t* err_word) {
@@ -310,7 +312,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         mbar_arrive(&bars->unit_full[slot]);
         if (u < 0) break;
         const UnitGeom g = unit_geom(p, u);
-        if (p.stream_flags != nullptr && g.zq / p.heads_per_piece != ready_piece) {
+        if (STREAMED && g.zq / p.heads_per_piece != ready_piece) {
           ready_piece = g.zq / p.heads_per_piece;
           if (!wait_piece_ready(p, ready_piece, bars, err_word)) break;
         }
@@ -757,7 +759,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
         if (p.lse != nullptr && row < p.N)
           p.lse[static_cast<int64_t>(g.zq) * p.N + row] =
               ((SCALED ? m : m * p.scale_log2) + (log2f(l) - p.log2_p_scale)) * 0.6931471805599453f;
-        if (p.stream_flags != nullptr) piece_tile_stored(p, g.zq, lane);
+        if constexpr (STREAMED) piece_tile_stored(p, g.zq, lane);
       }
       tc_fence_before();
       mbar_arrive(&bars->o_free[k]);
@@ -766,7 +768,7 @@ __global__ void __launch_bounds__(V2Config::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (p.stream_flags != nullptr && bars->abort && tid == 0) {
+  if (STREAMED && bars->abort && tid == 0) {
     // This CTA gave up: raise every piece flag, so that no copy stream waits
     // for outputs that will not come (the error word reports the failure).
     const int pieces = (p.B * p.H + p.heads_per_piece - 1) / p.heads_per_piece;
