@@ -255,7 +255,7 @@ int fp8attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, fl
  * aligned; lse_dev 4-byte aligned); their contents afterwards are those of
  * an fp8attn_fwd call on them.
  *
- * The problem is cut into `pieces` (1..16; 0 picks 12) pieces of whole
+ * The problem is cut into `pieces` (1..32; 0 picks the default) pieces of whole
  * (batch, kv head) slabs with their query heads.  Piece c's inputs are copied
  * on a copy stream of the library, which then sets a ready word; one
  * persistent kernel on `stream` processes the pieces in order, its producer
@@ -264,7 +264,7 @@ int fp8attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, fl
  * that piece's outputs back as soon as the flag is up.  The copy streams are
  * non-blocking streams the library creates once per device; the work on them
  * is joined back into `stream` before the call's later work.  The ready
- * words, flags and work-unit counter of a call sit in a 256-byte block of a
+ * words, flags and work-unit counter of a call sit in a 512-byte block of a
  * ring of eight that the library allocates once per device (stream memory
  * operations cannot address pool allocations); a block is reused only after
  * the stream of its previous call has passed that call's end.  Calls from
@@ -277,7 +277,7 @@ int fp8attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, fl
  * raises every flag (so no copy stream waits for good), the outputs are
  * undefined, and fp8attn_check_error() returns FP8ATTN_ERR_TIMEOUT.
  * Returns FP8ATTN_ERR_INVALID_ARG for a NULL host pointer, pieces outside
- * 0..16 or the checks of fp8attn_fwd (on the device buffers);
+ * 0..32 or the checks of fp8attn_fwd (on the device buffers);
  * FP8ATTN_ERR_UNSUPPORTED if the driver has no stream memory operations.
  */
 int fp8attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,

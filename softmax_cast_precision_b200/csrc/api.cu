@@ -355,7 +355,7 @@ StreamValueFn get_stream_value_fn(const char* name) {
 // fp8attn_fwd_host, made once.  The streams are non-blocking, so that they
 // never wait for the legacy default stream on which the kernel may be
 // running.  Stream memory operations reject stream-ordered (pool)
-// allocations, so the 256-byte blocks holding a call's work-unit counter,
+// allocations, so the 512-byte blocks holding a call's work-unit counter,
 // ready words and flags come from one cudaMalloc: a ring of kHostBlocks, each
 // handed to a new call only after the stream of its previous call has passed
 // the event recorded at that call's end.
@@ -364,7 +364,7 @@ struct HostStreams {
   cudaStream_t in = nullptr, out = nullptr;
   cudaEvent_t fork = nullptr, in_done = nullptr, out_done = nullptr;
   cudaEvent_t block_free[kHostBlocks] = {};
-  unsigned int* blocks = nullptr;  // kHostBlocks x 64 words
+  unsigned int* blocks = nullptr;  // kHostBlocks x kPieceBlockBytes
   int next = 0;
   StreamValueFn write32 = nullptr, wait32 = nullptr;
   bool ready = false;
@@ -386,7 +386,7 @@ int host_streams(HostStreams** out) {
         cudaEventCreateWithFlags(&h.fork, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&h.in_done, cudaEventDisableTiming) != cudaSuccess ||
         cudaEventCreateWithFlags(&h.out_done, cudaEventDisableTiming) != cudaSuccess ||
-        cudaMalloc(reinterpret_cast<void**>(&h.blocks), kHostBlocks * 256) != cudaSuccess)
+        cudaMalloc(reinterpret_cast<void**>(&h.blocks), kHostBlocks * kPieceBlockBytes) != cudaSuccess)
       return FP8ATTN_ERR_CUDA;
     for (int i = 0; i < kHostBlocks; ++i)
       if (cudaEventCreateWithFlags(&h.block_free[i], cudaEventDisableTiming) != cudaSuccess) return FP8ATTN_ERR_CUDA;
@@ -455,13 +455,13 @@ extern "C" int fp8attn_fwd_host(const void* q_host, const void* k_host, const vo
   const int n_pieces = static_cast<int>((zkv + kv_per_piece - 1) / kv_per_piece);
   const int rep = H / Hkv;
   p.heads_per_piece = kv_per_piece * rep;
-  // The 256-byte block holds the work-unit counter (word 0) and the piece words.
+  // The block holds the work-unit counter (word 0) and the piece words.
   const int slot = take_host_block(hs, s);
   if (slot < 0) return FP8ATTN_ERR_CUDA;
-  unsigned int* flags = hs->blocks + 64 * slot;
+  unsigned int* flags = hs->blocks + (kPieceBlockBytes / 4) * slot;
   const CUdeviceptr fl = reinterpret_cast<CUdeviceptr>(flags);
   p.stream_flags = flags;
-  bool ok = cudaMemsetAsync(flags, 0, 256, s) == cudaSuccess && cudaEventRecord(hs->fork, s) == cudaSuccess &&
+  bool ok = cudaMemsetAsync(flags, 0, kPieceBlockBytes, s) == cudaSuccess && cudaEventRecord(hs->fork, s) == cudaSuccess &&
             cudaStreamWaitEvent(hs->in, hs->fork, 0) == cudaSuccess &&
             cudaStreamWaitEvent(hs->out, hs->fork, 0) == cudaSuccess;
   // Copies in: each piece, then its ready word.
@@ -761,8 +761,8 @@ extern "C" int fp8attn_bwd(const void* q, const void* k, const void* v, const vo
     return FP8ATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   bwd_delta_kernel<<<static_cast<unsigned int>((rows + 7) / 8), 256, 0, s>>>(p);
-  bwd_dkdv_kernel<<<dim3(p.num_tiles, Hkv, B), 256, DkdvLayout::SMEM_BYTES, s>>>(tq, tk, tv, tdo, p, err_word);
-  bwd_dq_kernel<<<dim3(p.num_tiles, H, B), 256, DqLayout::SMEM_BYTES, s>>>(tq, tk, tv, tdo, p, err_word);
+  bwd_dkdv_kernel<<<dim3(p.num_tiles, Hkv, B), 128 * kBwdGroups, DkdvLayout::SMEM_BYTES, s>>>(tq, tk, tv, tdo, p, err_word);
+  bwd_dq_kernel<<<dim3(p.num_tiles, H, B), 128 * kBwdGroups, DqLayout::SMEM_BYTES, s>>>(tq, tk, tv, tdo, p, err_word);
   return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
 }
 

@@ -162,13 +162,14 @@ __device__ __forceinline__ void bwd_convert_row(const uint8_t* src, uint8_t* dst
   }
 }
 
-// Half of that: E4M3 columns 64 h .. 64 h + 63 of row `r` (h = 0, 1), so
-// that two threads share the conversion of a row.
-__device__ __forceinline__ void bwd_convert_half_row(const uint8_t* src, uint8_t* dst, int r, int h) {
+// Part h of that: E4M3 columns 16 NC h .. 16 NC (h + 1) - 1 of row `r`, so
+// that 8 / NC threads share the conversion of a row.
+template <int NC>
+__device__ __forceinline__ void bwd_convert_part_row(const uint8_t* src, uint8_t* dst, int r, int h) {
   const uint32_t s = smem_u32(src), d = smem_u32(dst);
 #pragma unroll
-  for (int cc = 0; cc < 4; ++cc) {
-    const int c = 4 * h + cc;
+  for (int cc = 0; cc < NC; ++cc) {
+    const int c = NC * h + cc;
     uint32_t w0, w1, w2, w3;
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
@@ -218,6 +219,11 @@ __device__ __forceinline__ float bwd_e4m3_value(float x) {
 //   bf16 tile, MN-major:    16 rows = 2048 bytes (+128); the N (or M) extent of
 //                           128 spans both panels, LBO = 16 KB apart.
 __device__ __forceinline__ uint64_t kmajor_desc(uint32_t saddr) { return smem_desc(saddr, 16, 1024, 2); }
+
+// Warpgroups of the two tensor-core backward kernels: each thread keeps one
+// TMEM lane (row) and takes 4 / kBwdGroups of the row's four 32-column chunks.
+constexpr int kBwdGroups = 4;
+constexpr int kBwdChunks = 4 / kBwdGroups;
 __device__ __forceinline__ uint64_t bf16_kmajor_step(int kk) {
   return static_cast<uint64_t>((kk >> 2) * (BwdConfig::BF_PANEL >> 4) + 2 * (kk & 3));
 }
@@ -249,7 +255,7 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const BwdParams p) {
 // --------------------------------------------------------------------------
 // dK and dV: one CTA (one warpgroup) per (batch, kv head, key tile).
 // --------------------------------------------------------------------------
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(128 * kBwdGroups, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const BwdParams p, uint32_t* err_word) {
@@ -267,8 +273,9 @@ __global__ void __launch_bounds__(256, 1)
   uint64_t* bar_drain = bars + 6;  // every product issued so far complete (abort path)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
 
-  // Two warpgroups: thread tid owns TMEM lane (key row) r = tid % 128 and, in
-  // each step, half wg = tid / 128 of the queries: chunks 2 wg and 2 wg + 1.
+  // kBwdGroups warpgroups: thread tid owns TMEM lane (key row) r = tid % 128
+  // and, in each step, part wg = tid / 128 of the queries (kBwdChunks chunks
+  // of 32).
   const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, r = tid & 127;
   const int jt = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int k0 = jt * 128;
@@ -340,22 +347,22 @@ __global__ void __launch_bounds__(256, 1)
 
   const int key = k0 + r;  // this thread's TMEM lane: one key
   bool fail = !mbar_wait_bounded(bar_kv, 0, err_word, kErrTimeoutKV);
-  if (!fail) bwd_convert_half_row(base + L::OFF_Q, base + L::OFF_VB, r, wg);
+  if (!fail) bwd_convert_part_row<8 / kBwdGroups>(base + L::OFF_Q, base + L::OFF_VB, r, wg);
   // Every thread has read V out of the Q buffer before Q_0 may overwrite it.
   fence_proxy_async_smem();
   bool abort = __syncthreads_or(fail) != 0;
   if (!abort && tid == 0 && n_iter > 0) issue_q(0);
   // lse (warpgroup 0) and D (warpgroup 1) of the step's 128 queries, fetched
-  // one step ahead.
+  // one step ahead (the other warpgroups fetch nothing).
   auto fetch_vec = [&](int it) -> float {
     float x = 0.0f;
-    if (it < n_iter) {
+    if (it < n_iter && wg < 2) {
       int zq, q0;
       step_geom(it, zq, q0);
       const int qi = q0 + r;
       if (qi < p.N) {
         const int64_t idx = static_cast<int64_t>(zq) * p.N + qi;
-        x = wg == 0 ? p.lse[idx] * 1.4426950408889634f : p.delta[idx];
+        x = (wg & 1) == 0 ? p.lse[idx] * 1.4426950408889634f : p.delta[idx];
       }
     }
     return x;
@@ -363,7 +370,7 @@ __global__ void __launch_bounds__(256, 1)
   float next_vec = fetch_vec(0);
 
   for (int it = 0; !abort && it < n_iter; ++it) {
-    (wg == 0 ? sLse2 : sDelta)[r] = next_vec;
+    if (wg < 2) ((wg & 1) == 0 ? sLse2 : sDelta)[r] = next_vec;
     next_vec = fetch_vec(it + 1);
     const uint32_t sDO = smem_u32(base + L::OFF_DO + (it & 1) * BwdConfig::BF_TILE);
     int zq, q0;
@@ -372,7 +379,7 @@ __global__ void __launch_bounds__(256, 1)
     if (!fail && tid == 0) q_landed = it + 1;
     if (!fail && !mbar_wait_bounded(bar_do + (it & 1), (it >> 1) & 1, err_word, kErrTimeoutQ)) fail = true;
     if (!fail && tid == 0) do_landed = it + 1;
-    if (!fail) bwd_convert_half_row(base + L::OFF_Q, base + L::OFF_QB, r, wg);
+    if (!fail) bwd_convert_part_row<8 / kBwdGroups>(base + L::OFF_Q, base + L::OFF_QB, r, wg);
     fence_proxy_async_smem();
     tc_fence_before();
     abort = __syncthreads_or(fail) != 0;
@@ -394,10 +401,10 @@ __global__ void __launch_bounds__(256, 1)
     // S^T(it) has read Q(it), which is converted already: fetch the next Q.
     if (tid == 0 && !fail && it + 1 < n_iter) issue_q(it + 1);
 
-    // P^T, E4M3(P^T S) and dS^T for this thread's key and half of the
+    // P^T, E4M3(P^T S) and dS^T for this thread's key and its part of the
     // queries, 32 at a time.
 #pragma unroll 1
-    for (int g = 2 * wg; g < 2 * wg + 2; ++g) {
+    for (int g = kBwdChunks * wg; g < kBwdChunks * (wg + 1); ++g) {
       uint32_t rs[32], rdp[32];
       tmem_ld32(tS + lane_off + 32 * g, rs);
       tmem_ld32(tDP + lane_off + 32 * g, rdp);
@@ -443,17 +450,20 @@ __global__ void __launch_bounds__(256, 1)
     // Warpgroup 0 writes dV / S, warpgroup 1 dK / sqrt(d).  Every lane takes
     // part in the warp-wide TMEM loads; lanes past N store nothing.
     const int64_t row = static_cast<int64_t>(zkv) * p.N + key;
-    float* dst = (wg == 0 ? p.dv : p.dk) + row * 128;
+    // Jobs j = 0..7: dV chunks 0..3, then dK chunks 0..3, spread over the warpgroups.
 #pragma unroll 1
-    for (int g = 0; g < 4; ++g) {
+    for (int job = wg * (8 / kBwdGroups); job < (wg + 1) * (8 / kBwdGroups); ++job) {
+      const bool is_dv = job < 4;
+      const int g = job & 3;
+      float* dst = (is_dv ? p.dv : p.dk) + row * 128;
       uint32_t a[32];
-      tmem_ld32((wg == 0 ? tDV : tDK) + lane_off + 32 * g, a);
+      tmem_ld32((is_dv ? tDV : tDK) + lane_off + 32 * g, a);
       tmem_wait_ld();
       if (key < p.N) {
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           float4 x;
-          if (wg == 0)
+          if (is_dv)
             x = make_float4(__fdiv_rn(__uint_as_float(a[e]), p.p_scale), __fdiv_rn(__uint_as_float(a[e + 1]), p.p_scale),
                             __fdiv_rn(__uint_as_float(a[e + 2]), p.p_scale), __fdiv_rn(__uint_as_float(a[e + 3]), p.p_scale));
           else
@@ -485,7 +495,7 @@ __global__ void __launch_bounds__(256, 1)
 // --------------------------------------------------------------------------
 // dQ: one CTA (one warpgroup) per (batch, head, query tile).
 // --------------------------------------------------------------------------
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(128 * kBwdGroups, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                   const BwdParams p, uint32_t* err_word) {
@@ -500,8 +510,9 @@ __global__ void __launch_bounds__(256, 1)
   uint64_t* bar_drain = bars + 4;  // every product issued so far complete (abort path)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 5);
 
-  // Two warpgroups: thread tid owns TMEM lane (query row) r = tid % 128 and,
-  // in each step, half wg = tid / 128 of the keys: chunks 2 wg and 2 wg + 1.
+  // kBwdGroups warpgroups: thread tid owns TMEM lane (query row) r = tid % 128
+  // and, in each step, part wg = tid / 128 of the keys (kBwdChunks chunks of
+  // 32).
   const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, r = tid & 127;
   const int it_q = p.num_tiles - 1 - static_cast<int>(blockIdx.x);  // longest causal rows first
   const int h = blockIdx.y, b = blockIdx.z;
@@ -563,11 +574,12 @@ __global__ void __launch_bounds__(256, 1)
     if (!fail && !mbar_wait_bounded(bar_kv, j & 1, err_word, kErrTimeoutKV)) fail = true;
     if (!fail && tid == 0) kv_landed = j + 1;
     if (!fail) {
-      // Warpgroup 0 converts K, warpgroup 1 V.
-      if (wg == 0)
-        bwd_convert_row(base + L::OFF_K, base + L::OFF_KB + (j & 1) * BwdConfig::BF_TILE, r);
+      // The first half of the warpgroups converts K, the second half V.
+      constexpr int kHalf = kBwdGroups / 2;
+      if (wg < kHalf)
+        bwd_convert_part_row<8 / kHalf>(base + L::OFF_K, base + L::OFF_KB + (j & 1) * BwdConfig::BF_TILE, r, wg);
       else
-        bwd_convert_row(base + L::OFF_V, base + L::OFF_VB, r);
+        bwd_convert_part_row<8 / kHalf>(base + L::OFF_V, base + L::OFF_VB, r, wg - kHalf);
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -594,7 +606,7 @@ __global__ void __launch_bounds__(256, 1)
     // dS is single-buffered: the previous step's dQ product must have read it.
     if (j > 0 && !mbar_wait_bounded(bar_g, (j - 1) & 1, err_word, kErrTimeoutMMA)) fail = true;
 #pragma unroll 1
-    for (int g = 2 * wg; g < 2 * wg + 2; ++g) {
+    for (int g = kBwdChunks * wg; g < kBwdChunks * (wg + 1); ++g) {
       uint32_t rs[32], rdp[32];
       tmem_ld32(tS + lane_off + 32 * g, rs);
       tmem_ld32(tDP + lane_off + 32 * g, rdp);
@@ -634,7 +646,7 @@ __global__ void __launch_bounds__(256, 1)
   if (!abort) {
     float* dqrow = p.dq + ridx * 128;
 #pragma unroll 1
-    for (int g = 2 * wg; g < 2 * wg + 2; ++g) {
+    for (int g = kBwdChunks * wg; g < kBwdChunks * (wg + 1); ++g) {
       uint32_t a[32];
       tmem_ld32(tDQ + lane_off + 32 * g, a);
       tmem_wait_ld();

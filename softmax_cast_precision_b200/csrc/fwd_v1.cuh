@@ -58,12 +58,13 @@ struct FwdParams {
   int heads_per_piece;
 };
 
-// Word offsets in FwdParams::stream_flags (word 0 is the work-unit counter
-// when the same block holds both).
-constexpr int kPieceReady = 16;
-constexpr int kPieceDone = 32;
-constexpr int kPieceFlag = 48;
-constexpr int kMaxPieces = 16;
+// Word offsets in FwdParams::stream_flags, a 512-byte block (word 0 is the
+// work-unit counter when the same block holds both).
+constexpr int kMaxPieces = 32;
+constexpr int kPieceReady = 32;
+constexpr int kPieceDone = 64;
+constexpr int kPieceFlag = 96;
+constexpr int kPieceBlockBytes = 512;
 
 template <int D>
 struct V1Config {

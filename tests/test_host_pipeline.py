@@ -22,7 +22,7 @@ def _call_host(fp8, pieces=0, qh=16, kh=16, vh=16, oh=16, lh=16, qd=16, kd=16, v
 
 
 @pytest.mark.parametrize("kw,expected", [
-    (dict(pieces=-1), 1), (dict(pieces=17), 1), (dict(qh=0), 1), (dict(kh=0), 1), (dict(vh=0), 1), (dict(oh=0), 1),
+    (dict(pieces=-1), 1), (dict(pieces=33), 1), (dict(qh=0), 1), (dict(kh=0), 1), (dict(vh=0), 1), (dict(oh=0), 1),
     (dict(od=0), 1), (dict(od=8), 1), (dict(qd=0), 1), (dict(ld=0), 1), (dict(lh=0), 1), (dict(ld=18), 1),
     (dict(d=96), 2), (dict(H=3), 1), (dict(N=0), 0), (dict(N=0, qh=0, qd=0, kd=0, vd=0), 0),
 ])
