@@ -255,20 +255,23 @@ int fp8attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, fl
  * aligned; lse_dev 4-byte aligned); their contents afterwards are those of
  * an fp8attn_fwd call on them.
  *
- * The problem is cut into `pieces` (1..32; 0 picks the default) pieces of whole
- * (batch, kv head) slabs with their query heads.  Piece c's inputs are copied
- * on a copy stream of the library, which then sets a ready word; one
- * persistent kernel on `stream` processes the pieces in order, its producer
- * waiting for each piece's ready word; as the last query tile of a piece is
- * stored the kernel raises the piece's flag, and a second copy stream copies
- * that piece's outputs back as soon as the flag is up.  The copy streams are
- * non-blocking streams the library creates once per device; the work on them
- * is joined back into `stream` before the call's later work.  The ready
- * words, flags and work-unit counter of a call sit in a 512-byte block of a
- * ring of eight that the library allocates once per device (stream memory
- * operations cannot address pool allocations); a block is reused only after
- * the stream of its previous call has passed that call's end.  Calls from
- * several host threads on one device must be ordered by the caller.
+ * The problem is cut into `pieces` (1..32; 0 picks 24; never more than the
+ * number of (batch, kv head) slabs) pieces of whole (batch, kv head) slabs
+ * with their query heads.  The inputs are copied on a copy stream of the
+ * library, in runs of neighbouring pieces (one piece first, then two, then
+ * three at a time, then two and one at the end), each run followed by the
+ * ready words of its pieces.  One persistent kernel on `stream` processes the
+ * pieces in order, its producer waiting for each piece's ready word; as the
+ * last query tile of a piece is stored the kernel raises the piece's flag, and
+ * a second copy stream copies each run's outputs back once the flags of all
+ * its pieces are up.  The copy streams are non-blocking streams the library
+ * creates once per device; the work on them is joined back into `stream`
+ * before the call's later work.  The ready words, flags and work-unit counter
+ * of a call sit in a 512-byte block of a ring of eight that the library
+ * allocates once per device (stream memory operations cannot address pool
+ * allocations); a block is reused only after the stream of its previous call
+ * has passed that call's end.  Calls from several host threads on one device
+ * must be ordered by the caller.
  * With d = 64 or pieces = 1 the copies in, the pass and the copies out simply
  * run in order on `stream`.
  *

@@ -449,12 +449,36 @@ extern "C" int fp8attn_fwd_host(const void* q_host, const void* k_host, const vo
   HostStreams* hs = nullptr;
   st = host_streams(&hs);
   if (st != FP8ATTN_OK) return st;
-  // Pieces of whole (b, kv head) slabs with their query heads.
-  const int want = pieces == 0 ? 12 : pieces;
+  // Pieces of whole (b, kv head) slabs with their query heads: the units the
+  // pass waits for and reports.
+  const int want = pieces == 0 ? 24 : pieces;
   const int kv_per_piece = static_cast<int>((zkv + want - 1) / want);
   const int n_pieces = static_cast<int>((zkv + kv_per_piece - 1) / kv_per_piece);
   const int rep = H / Hkv;
   p.heads_per_piece = kv_per_piece * rep;
+  // Copies move runs of neighbouring pieces: one piece first (so that the pass
+  // starts early), then two, then three at a time, then two and one last (so
+  // that little is left to compute and copy out after the last copy in).
+  // Fewer, larger copies keep the host link busy; short ones at both ends
+  // shorten the time when only one direction of it is in use.
+  int group_end[kMaxPieces];
+  int n_groups = 0;
+  {
+    int c = 0;
+    auto add = [&](int len) {
+      c += len;
+      group_end[n_groups++] = c;
+    };
+    if (n_pieces < 6) {
+      for (int i = 0; i < n_pieces; ++i) add(1);
+    } else {
+      add(1);
+      add(2);
+      for (int mid = n_pieces - 6; mid > 0; mid -= std::min(3, mid)) add(std::min(3, mid));
+      add(2);
+      add(1);
+    }
+  }
   // The block holds the work-unit counter (word 0) and the piece words.
   const int slot = take_host_block(hs, s);
   if (slot < 0) return FP8ATTN_ERR_CUDA;
@@ -464,15 +488,21 @@ extern "C" int fp8attn_fwd_host(const void* q_host, const void* k_host, const vo
   bool ok = cudaMemsetAsync(flags, 0, kPieceBlockBytes, s) == cudaSuccess && cudaEventRecord(hs->fork, s) == cudaSuccess &&
             cudaStreamWaitEvent(hs->in, hs->fork, 0) == cudaSuccess &&
             cudaStreamWaitEvent(hs->out, hs->fork, 0) == cudaSuccess;
-  // Copies in: each piece, then its ready word.
-  for (int c = 0; ok && c < n_pieces; ++c) {
-    const size_t k0 = static_cast<size_t>(c) * kv_per_piece;
-    const size_t nk = std::min<size_t>(kv_per_piece, zkv - k0);
+  // Slabs of the pieces [c0, c1): kv slabs [k0, k0 + nk), query slabs [k0, k0 + nk) * rep.
+  auto slabs = [&](int c0, int c1, size_t& k0, size_t& nk) {
+    k0 = static_cast<size_t>(c0) * kv_per_piece;
+    nk = std::min<size_t>(static_cast<size_t>(c1) * kv_per_piece, zkv) - k0;
+  };
+  // Copies in: each run, then the ready words of its pieces.
+  for (int g = 0, c0 = 0; ok && g < n_groups; c0 = group_end[g++]) {
+    size_t k0, nk;
+    slabs(c0, group_end[g], k0, nk);
     const size_t q0 = k0 * rep, nq = nk * rep;
     ok = h2d(static_cast<uint8_t*>(q_dev) + q0 * row, static_cast<const uint8_t*>(q_host) + q0 * row, nq * row, hs->in) &&
          h2d(static_cast<uint8_t*>(k_dev) + k0 * row, static_cast<const uint8_t*>(k_host) + k0 * row, nk * row, hs->in) &&
-         h2d(static_cast<uint8_t*>(v_dev) + k0 * row, static_cast<const uint8_t*>(v_host) + k0 * row, nk * row, hs->in) &&
-         hs->write32(reinterpret_cast<CUstream>(hs->in), fl + 4 * (kPieceReady + c), 1u, 0) == CUDA_SUCCESS;
+         h2d(static_cast<uint8_t*>(v_dev) + k0 * row, static_cast<const uint8_t*>(v_host) + k0 * row, nk * row, hs->in);
+    for (int c = c0; ok && c < group_end[g]; ++c)
+      ok = hs->write32(reinterpret_cast<CUstream>(hs->in), fl + 4 * (kPieceReady + c), 1u, 0) == CUDA_SUCCESS;
   }
   // (Recorded whatever happened above, so that the join below also covers
   // copies and ready words queued before a failure.)
@@ -482,15 +512,20 @@ extern "C" int fp8attn_fwd_host(const void* q_host, const void* k_host, const vo
   // returns only when done, and must not wait for a kernel not yet launched.
   if (ok) st = launch_v2_on<false>(q_dev, k_dev, v_dev, p, s, flags);
   if (!ok && st == FP8ATTN_OK) st = FP8ATTN_ERR_CUDA;
-  // Copies out: each piece once its flag is up (the kernel raises every flag,
-  // also when it gives up, so these waits always end once it has run).
-  for (int c = 0; st == FP8ATTN_OK && c < n_pieces; ++c) {
-    const size_t q0 = static_cast<size_t>(c) * p.heads_per_piece;
-    const size_t nq = std::min<size_t>(p.heads_per_piece, zq - q0);
-    if (hs->wait32(reinterpret_cast<CUstream>(hs->out), fl + 4 * (kPieceFlag + c), 1u, 0 /* GEQ */) != CUDA_SUCCESS ||
-        !d2h(static_cast<uint8_t*>(o_host) + q0 * row * 2, static_cast<const uint8_t*>(o_dev) + q0 * row * 2,
-             nq * row * 2, hs->out) ||
-        (lse_dev && !d2h(lse_host + q0 * N, lse_dev + q0 * N, nq * N * sizeof(float), hs->out)))
+  // Copies out: each run once the flags of all its pieces are up (the kernel
+  // raises every flag, also when it gives up, so these waits always end once
+  // it has run).
+  for (int g = 0, c0 = 0; st == FP8ATTN_OK && g < n_groups; c0 = group_end[g++]) {
+    for (int c = c0; st == FP8ATTN_OK && c < group_end[g]; ++c)
+      if (hs->wait32(reinterpret_cast<CUstream>(hs->out), fl + 4 * (kPieceFlag + c), 1u, 0 /* GEQ */) != CUDA_SUCCESS)
+        st = FP8ATTN_ERR_CUDA;
+    size_t k0, nk;
+    slabs(c0, group_end[g], k0, nk);
+    const size_t q0 = k0 * rep, nq = nk * rep;
+    if (st == FP8ATTN_OK &&
+        (!d2h(static_cast<uint8_t*>(o_host) + q0 * row * 2, static_cast<const uint8_t*>(o_dev) + q0 * row * 2,
+              nq * row * 2, hs->out) ||
+         (lse_dev && !d2h(lse_host + q0 * N, lse_dev + q0 * N, nq * N * sizeof(float), hs->out))))
       st = FP8ATTN_ERR_CUDA;
   }
   // Join: the stream continues once the copies out (and in) are done; the
