@@ -50,3 +50,41 @@ def test_wait_runs_out_and_the_next_call_is_correct(fp8, counting):
     vmax = float(np.abs(oracle.e4m3_decode(v)).max())
     assert float(np.abs(o.float().cpu().numpy() - ref.o).max()) <= 1e-2 * vmax
     assert float(np.abs(lse.cpu().numpy() - ref.lse).max()) <= 1e-3
+
+
+_STREAMED_CHILD = r"""
+import sys
+sys.path.insert(0, {root!r})
+import torch
+import synthetic
+from softmax_cast_precision_b200 import fp8attn as fp8
+q, k, v, _ = synthetic.make_inputs(1, 8, 4, 1000, 128, 7.0, seed=93)
+qh, kh, vh = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
+fp8.check_error()
+fp8.test_withhold_load(20_000_000)  # 20 ms
+fp8.fwd_host(qh, kh, vh, causal=True, pieces=4)  # returns: every piece flag is raised by the CTAs that gave up
+try:
+    fp8.check_error()
+    sys.exit("no timeout reported")
+except fp8.Fp8AttnError as e:
+    assert e.status == fp8.ERR_TIMEOUT, e.status
+o_h, l_h = fp8.fwd_host(qh, kh, vh, causal=True, pieces=4)
+fp8.check_error()
+o_ref, l_ref = fp8.fwd(qh.cuda(), kh.cuda(), vh.cuda(), causal=True)
+assert torch.equal(o_h, o_ref.cpu()) and torch.equal(l_h, l_ref.cpu())
+print("ok")
+"""
+
+
+def test_streamed_call_returns_after_a_wait_runs_out(fp8):
+    """fp8attn_fwd_host with a wait made to run out: the kernel raises every piece flag as it gives up, so the
+    copy-out stream's waits end and the call returns; the next call matches fwd bit for bit.  Run in a child
+    process with a time limit, so that a regression shows as a failure rather than a stuck test run."""
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    res = subprocess.run([sys.executable, "-c", _STREAMED_CHILD.format(root=root)], cwd=root, timeout=180,
+                         capture_output=True, text=True)
+    assert res.returncode == 0 and res.stdout.strip().endswith("ok"), res.stdout + res.stderr
