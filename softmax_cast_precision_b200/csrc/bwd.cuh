@@ -202,12 +202,25 @@ __device__ __forceinline__ void bwd_store_bf16_32(uint8_t* dst, int r, int g, co
   }
 }
 
-// The E4M3 value nearest to x (nearest even, saturating), as float32.
-__device__ __forceinline__ float bwd_e4m3_value(float x) {
-  const uint32_t code = cvt_e4m3x2(x, 0.0f);
+// bfloat16 pair (lo in the low half) of the E4M3 values nearest to lo and
+// hi (nearest even, saturating): exact, every E4M3 value being a bfloat16.
+__device__ __forceinline__ uint32_t bwd_e4m3_pair_bf16(float lo, float hi) {
+  const uint32_t code = cvt_e4m3x2(lo, hi);
   uint32_t h;
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(code)));
-  return __low2float(*reinterpret_cast<const __half2*>(&h));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return pack_bf16x2(f.x, f.y);
+}
+
+// Stores 32 values already packed as 16 bfloat16 pairs (columns 32 g ..
+// 32 g + 31 of row `r`) as chunks 4g .. 4g+3 of a two-panel tile.
+__device__ __forceinline__ void bwd_store_bf16_packed(uint8_t* dst, int r, int g, const uint32_t (&w)[16]) {
+  const uint32_t d = smem_u32(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d + bf16_tile_chunk(r, 4 * g + q)), "r"(w[4 * q]),
+                 "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
+                 : "memory");
 }
 
 // Descriptors of the three operand forms (start address, LBO, SBO, 128-byte
@@ -362,7 +375,7 @@ __global__ void __launch_bounds__(128 * kBwdGroups, 1)
       const int qi = q0 + r;
       if (qi < p.N) {
         const int64_t idx = static_cast<int64_t>(zq) * p.N + qi;
-        x = (wg & 1) == 0 ? p.lse[idx] * 1.4426950408889634f : p.delta[idx];
+        x = (wg & 1) == 0 ? p.lse[idx] : p.delta[idx];  // used one step later
       }
     }
     return x;
@@ -370,7 +383,8 @@ __global__ void __launch_bounds__(128 * kBwdGroups, 1)
   float next_vec = fetch_vec(0);
 
   for (int it = 0; !abort && it < n_iter; ++it) {
-    if (wg < 2) ((wg & 1) == 0 ? sLse2 : sDelta)[r] = next_vec;
+    if (wg == 0) sLse2[r] = next_vec * 1.4426950408889634f;  // lse in log2 units
+    if (wg == 1) sDelta[r] = next_vec;
     next_vec = fetch_vec(it + 1);
     const uint32_t sDO = smem_u32(base + L::OFF_DO + (it & 1) * BwdConfig::BF_TILE);
     int zq, q0;
@@ -403,23 +417,37 @@ __global__ void __launch_bounds__(128 * kBwdGroups, 1)
 
     // P^T, E4M3(P^T S) and dS^T for this thread's key and its part of the
     // queries, 32 at a time.
+    // Only tiles on the diagonal or past N mask any (key, query) pair.
+    const bool edge = q0 + 128 > p.N || k0 + 128 > p.N || (p.causal && k0 + 127 > q0);
 #pragma unroll 1
     for (int g = kBwdChunks * wg; g < kBwdChunks * (wg + 1); ++g) {
       uint32_t rs[32], rdp[32];
       tmem_ld32(tS + lane_off + 32 * g, rs);
       tmem_ld32(tDP + lane_off + 32 * g, rdp);
       tmem_wait_ld();
-      float ph[32], ds[32];
+      uint32_t php[16];
+      float ds[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const int c = 32 * g + e;
-        const int qi = q0 + c;
-        const bool visible = qi < p.N && key < p.N && (!p.causal || key <= qi);
-        const float pr = visible ? ex2_approx(__uint_as_float(rs[e]) * p.scale_log2 - sLse2[c]) : 0.0f;
-        ph[e] = bwd_e4m3_value(pr * p.p_scale);
-        ds[e] = pr * (__uint_as_float(rdp[e]) - sDelta[c]);
+      for (int e4 = 0; e4 < 8; ++e4) {
+        const float4 lv = reinterpret_cast<const float4*>(sLse2 + 32 * g)[e4];
+        const float4 dv = reinterpret_cast<const float4*>(sDelta + 32 * g)[e4];
+        const float la[4] = {lv.x, lv.y, lv.z, lv.w}, da[4] = {dv.x, dv.y, dv.z, dv.w};
+        float pr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int e = 4 * e4 + i;
+          pr[i] = ex2_approx(__uint_as_float(rs[e]) * p.scale_log2 - la[i]);
+          if (edge) {
+            const int qi = q0 + 32 * g + e;
+            const bool visible = qi < p.N && key < p.N && (!p.causal || key <= qi);
+            pr[i] = visible ? pr[i] : 0.0f;
+          }
+          ds[e] = pr[i] * (__uint_as_float(rdp[e]) - da[i]);
+        }
+        php[2 * e4] = bwd_e4m3_pair_bf16(pr[0] * p.p_scale, pr[1] * p.p_scale);
+        php[2 * e4 + 1] = bwd_e4m3_pair_bf16(pr[2] * p.p_scale, pr[3] * p.p_scale);
       }
-      bwd_store_bf16_32(base + L::OFF_PT, r, g, ph);
+      bwd_store_bf16_packed(base + L::OFF_PT, r, g, php);
       bwd_store_bf16_32(base + L::OFF_DST, r, g, ds);
     }
     fence_proxy_async_smem();
@@ -603,6 +631,8 @@ __global__ void __launch_bounds__(128 * kBwdGroups, 1)
     // the barrier): fetch the next key tile while this one is finished.
     if (tid == 0 && !fail && j < last) issue_kv(j + 1);
 
+    // Only tiles on the diagonal or past N mask any (query, key) pair.
+    const bool edge = q0 + 128 > p.N || j0 + 128 > p.N || (p.causal && j0 + 127 > q0);
     // dS is single-buffered: the previous step's dQ product must have read it.
     if (j > 0 && !mbar_wait_bounded(bar_g, (j - 1) & 1, err_word, kErrTimeoutMMA)) fail = true;
 #pragma unroll 1
@@ -614,9 +644,12 @@ __global__ void __launch_bounds__(128 * kBwdGroups, 1)
       float ds[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const int kj = j0 + 32 * g + e;
-        const bool visible = row < p.N && kj < p.N && (!p.causal || kj <= row);
-        const float pr = visible ? ex2_approx(__uint_as_float(rs[e]) * p.scale_log2 - lse2) : 0.0f;
+        float pr = ex2_approx(__uint_as_float(rs[e]) * p.scale_log2 - lse2);
+        if (edge) {
+          const int kj = j0 + 32 * g + e;
+          const bool visible = row < p.N && kj < p.N && (!p.causal || kj <= row);
+          pr = visible ? pr : 0.0f;
+        }
         ds[e] = pr * (__uint_as_float(rdp[e]) - dlt);
       }
       bwd_store_bf16_32(base + L::OFF_DS, r, g, ds);
