@@ -65,12 +65,14 @@ __device__ __forceinline__ int quant_scale_exponent(float amax) {
   return e < -126 ? -126 : e;
 }
 
-// One thread's E elements of a row, read from the staged block: chunk c
-// (elements 8c .. 8c + 7 of the thread's list) is row element 32 c + 8 part.
-// Rows past the block's end read as zeros.
+// One thread's E elements of a row, read from the staged block: slot c
+// (elements 8c .. 8c + 7 of the thread's list) holds chunk c ^ sw, row
+// elements 32 (c ^ sw) + 8 part ..  With sw = 1 on odd rows, the two rows of
+// a quarter-warp read opposite 64-byte halves of their 256-byte rows, so the
+// 16-byte reads hit distinct banks.  Rows past the block's end read as zeros.
 template <int E>
 __device__ __forceinline__ void quant_read_row(const uint8_t* stage, int row_bytes, int r, int rows, int part,
-                                               int x_f32, const uint4* sign_masks, float (&v)[E]) {
+                                               int x_f32, const uint4* sign_masks, int sw, float (&v)[E]) {
   if (r >= rows) {
 #pragma unroll
     for (int e = 0; e < E; ++e) v[e] = 0.0f;
@@ -80,8 +82,8 @@ __device__ __forceinline__ void quant_read_row(const uint8_t* stage, int row_byt
     const float* src = reinterpret_cast<const float*>(stage + static_cast<int64_t>(r) * row_bytes) + 8 * part;
 #pragma unroll
     for (int c = 0; c < E / 8; ++c) {
-      const float4 a = *reinterpret_cast<const float4*>(src + 32 * c);
-      const float4 b = *reinterpret_cast<const float4*>(src + 32 * c + 4);
+      const float4 a = *reinterpret_cast<const float4*>(src + 32 * (c ^ sw));
+      const float4 b = *reinterpret_cast<const float4*>(src + 32 * (c ^ sw) + 4);
       v[8 * c + 0] = a.x; v[8 * c + 1] = a.y; v[8 * c + 2] = a.z; v[8 * c + 3] = a.w;
       v[8 * c + 4] = b.x; v[8 * c + 5] = b.y; v[8 * c + 6] = b.z; v[8 * c + 7] = b.w;
     }
@@ -90,9 +92,9 @@ __device__ __forceinline__ void quant_read_row(const uint8_t* stage, int row_byt
     const uint16_t* src = reinterpret_cast<const uint16_t*>(stage + static_cast<int64_t>(r) * row_bytes) + 8 * part;
 #pragma unroll
     for (int c = 0; c < E / 8; ++c) {
-      const uint4 q = *reinterpret_cast<const uint4*>(src + 32 * c);
+      const uint4 q = *reinterpret_cast<const uint4*>(src + 32 * (c ^ sw));
       // With a rotation, the signs flip the bfloat16 sign bits (bits 15 and 31 of each word).
-      const uint4 sm = sign_masks ? sign_masks[c * kQuantThreadsPerRow + part] : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 sm = sign_masks ? sign_masks[(c ^ sw) * kQuantThreadsPerRow + part] : make_uint4(0u, 0u, 0u, 0u);
       const uint32_t w[4] = {q.x ^ sm.x, q.y ^ sm.y, q.z ^ sm.z, q.w ^ sm.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -126,11 +128,32 @@ __device__ __forceinline__ void quant_stage(float (&v)[E]) {
   }
 }
 
+// The stage of half-width 32 (slot bit 0) when slots 2i and 2i + 1 may hold
+// chunks 2i + 1 and 2i (sw = 1): the member in slot 2i is then the upper
+// one.  new slot 2i = s1 * slot 2i + slot 2i+1, new slot 2i+1 = s2 * slot
+// 2i+1 + slot 2i, with (s1, s2) = (1, -1) or (-1, 1): a sum or a difference,
+// one rounding each, exactly as in the unswapped order.
+template <int E>
+__device__ __forceinline__ void quant_stage32(float (&v)[E], int sw) {
+  const float s1 = sw ? -1.0f : 1.0f;
+  const uint64_t sg1 = f2_pack(s1, s1), sg2 = f2_pack(-s1, -s1);
+#pragma unroll
+  for (int e = 0; e < E; e += 2) {
+    if ((e & 8) == 0) {
+      const uint64_t a = f2_pack(v[e], v[e + 1]), b = f2_pack(v[e + 8], v[e + 9]);
+      f2_unpack(f2_fma(a, sg1, b), v[e], v[e + 1]);
+      f2_unpack(f2_fma(b, sg2, a), v[e + 8], v[e + 9]);
+    }
+  }
+}
+
 // The signs and the unnormalised transform x H_d over the thread's E values
 // (the factor 1/sqrt(d) is applied by the caller).  sb[c] holds the 8 sign
-// bits of chunk c (bit j set: element j of the chunk is negated).
+// bits of chunk c (bit j set: element j of the chunk is negated); they are
+// applied here only when not already applied to the raw words (and then the
+// slots are not swapped, sw = 0).
 template <int E>
-__device__ __forceinline__ void quant_rotate_row(int part, const uint32_t (&sb)[E / 8], bool signs_applied,
+__device__ __forceinline__ void quant_rotate_row(int part, const uint32_t (&sb)[E / 8], bool signs_applied, int sw,
                                                  float (&v)[E]) {
   if (!signs_applied) {
 #pragma unroll
@@ -155,16 +178,16 @@ __device__ __forceinline__ void quant_rotate_row(int part, const uint32_t (&sb)[
     }
   }
   // Half-widths 32 and 64: chunk bits of the thread's list (8 and 16 in it).
-  quant_stage<E, 8>(v);
+  quant_stage32<E>(v, sw);
   if constexpr (E > 16) quant_stage<E, 16>(v);
 }
 
 // Stores E4M3(v * mul): mul = c / s, with c = float32(1/sqrt(d)) after a
 // rotation (else 1) and s the block's power-of-two descale, so that
-// v * mul = (v * c) / s exactly (s is a power of two).  Chunk c goes to row
-// bytes 32 c + 8 part .. + 7.
+// v * mul = (v * c) / s exactly (s is a power of two).  Slot c (chunk c ^ sw)
+// goes to row bytes 32 (c ^ sw) + 8 part .. + 7.
 template <int E>
-__device__ __forceinline__ void quant_store_row(uint8_t* dst_row, int part, const float (&v)[E], float mul) {
+__device__ __forceinline__ void quant_store_row(uint8_t* dst_row, int part, const float (&v)[E], float mul, int sw) {
   const uint64_t m2 = f2_pack(mul, mul);
 #pragma unroll
   for (int c = 0; c < E / 8; ++c) {
@@ -177,7 +200,7 @@ __device__ __forceinline__ void quant_store_row(uint8_t* dst_row, int part, cons
       f2_unpack(f2_mul(f2_pack(v[e + 2], v[e + 3]), m2), cc, dd);
       w[j] = cvt_e4m3x4(a, b, cc, dd);
     }
-    *reinterpret_cast<uint2*>(dst_row + 32 * c + 8 * part) = make_uint2(w[0], w[1]);
+    *reinterpret_cast<uint2*>(dst_row + 32 * (c ^ sw) + 8 * part) = make_uint2(w[0], w[1]);
   }
 }
 
@@ -254,6 +277,9 @@ __global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const Qua
   // (positive scaling is monotone, so max |v c| = max|v| c) and folded into
   // the cast's multiplier.
   const float cnorm = p.rotate ? ((E == 32) ? 0.08838834764831845f : 0.125f) : 1.0f;
+  // Odd rows hold their chunk pairs swapped (bfloat16 inputs; see quant_read_row).
+  // Every row this thread handles has the parity of rsub (rows rsub + 64 i).
+  const int sw = p.x_f32 ? 0 : (rsub & 1);
 
   int k = 0;
   bool aborted = false;
@@ -270,8 +296,8 @@ __global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const Qua
       // Every lane transforms (rows past the block's end hold zeros), so the
       // full-warp shuffles of the rotation always have all 32 lanes.
       quant_read_row<E>(stage, row_bytes, rsub + i * kQuantRowsPerPass, ok ? rows : 0, part, p.x_f32,
-                        word_signs ? sign_masks : nullptr, v[i]);
-      if (p.rotate) quant_rotate_row<E>(part, sb, word_signs, v[i]);
+                        word_signs ? sign_masks : nullptr, sw, v[i]);
+      if (p.rotate) quant_rotate_row<E>(part, sb, word_signs, sw, v[i]);
 #pragma unroll
       for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(v[i][e]));
     }
@@ -305,7 +331,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const Qua
 #pragma unroll
     for (int i = 0; i < kPasses; ++i) {
       const int r = rsub + i * kQuantRowsPerPass;
-      if (r < rows) quant_store_row<E>(p.xq + (static_cast<int64_t>(z) * p.N + r0 + r) * p.d, part, v[i], mul);
+      if (r < rows) quant_store_row<E>(p.xq + (static_cast<int64_t>(z) * p.N + r0 + r) * p.d, part, v[i], mul, sw);
     }
   }
   // After a wait ran out: let the copies still in flight land before the CTA's
