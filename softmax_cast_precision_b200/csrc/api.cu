@@ -782,9 +782,10 @@ extern "C" int fp8attn_bwd(const void* q, const void* k, const void* v, const vo
   p.p_scale = p_scale;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
   p.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(128.0));
-  CUtensorMap tq, tk, tv, tdo;
-  if (!make_map(&tq, q, 128, N, B * H, 128) || !make_map(&tk, k, 128, N, B * Hkv, 128) ||
-      !make_map(&tv, v, 128, N, B * Hkv, 128) || !make_map_bf16(&tdo, dout, N, B * H))
+  CUtensorMap tq, tq64, tk, tv, tdo;
+  if (!make_map(&tq, q, 128, N, B * H, 128) || !make_map(&tq64, q, 128, N, B * H, 64) ||
+      !make_map(&tk, k, 128, N, B * Hkv, 128) || !make_map(&tv, v, 128, N, B * Hkv, 128) ||
+      !make_map_bf16(&tdo, dout, N, B * H))
     return FP8ATTN_ERR_CUDA;
   uint32_t* err_word = nullptr;
   if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err_word), g_error_word) != cudaSuccess)
@@ -796,7 +797,8 @@ extern "C" int fp8attn_bwd(const void* q, const void* k, const void* v, const vo
     return FP8ATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   bwd_delta_kernel<<<static_cast<unsigned int>((rows + 7) / 8), 256, 0, s>>>(p);
-  bwd_dkdv_kernel<<<dim3(p.num_tiles, Hkv, B), 128 * kBwdGroups, DkdvLayout::SMEM_BYTES, s>>>(tq, tk, tv, tdo, p, err_word);
+  bwd_dkdv_kernel<<<dim3(p.num_tiles, Hkv, B), kDkdvThreads, DkdvLayout::SMEM_BYTES, s>>>(tq64, tk, tv, tdo, p,
+                                                                                        err_word);
   bwd_dq_kernel<<<dim3(p.num_tiles, H, B), 128 * kBwdGroups, DqLayout::SMEM_BYTES, s>>>(tq, tk, tv, tdo, p, err_word);
   return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
 }

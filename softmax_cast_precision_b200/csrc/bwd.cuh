@@ -82,7 +82,7 @@ struct DkdvLayout {
   static constexpr int OFF_DST = OFF_PT + BwdConfig::BF_TILE;       // dS^T  bf16
   static constexpr int OFF_VEC = OFF_DST + BwdConfig::BF_TILE;      // lse_i * log2(e) [128], D_i [128]
   static constexpr int OFF_BAR = OFF_VEC + 2 * 128 * 4;
-  static constexpr int SMEM_BYTES = OFF_BAR + 128 + 1024;           // barriers, TMEM slot, alignment slack
+  static constexpr int SMEM_BYTES = OFF_BAR + 192 + 1024;           // barriers, TMEM slot, alignment slack
 };
 
 // Shared-memory layout of bwd_dq_kernel.
@@ -223,6 +223,26 @@ __device__ __forceinline__ void bwd_store_bf16_packed(uint8_t* dst, int r, int g
                  : "memory");
 }
 
+// 16 values (columns 8 c0 .. 8 c0 + 15 of row `r`) as bfloat16 chunks c0 and
+// c0 + 1 of a two-panel tile: from FP32 values, or already packed in pairs.
+__device__ __forceinline__ void bwd_store_bf16_16(uint8_t* dst, int r, int c0, const float (&x)[16]) {
+  const uint32_t d = smem_u32(dst);
+#pragma unroll
+  for (int q = 0; q < 2; ++q)
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d + bf16_tile_chunk(r, c0 + q)),
+                 "r"(pack_bf16x2(x[8 * q + 0], x[8 * q + 1])), "r"(pack_bf16x2(x[8 * q + 2], x[8 * q + 3])),
+                 "r"(pack_bf16x2(x[8 * q + 4], x[8 * q + 5])), "r"(pack_bf16x2(x[8 * q + 6], x[8 * q + 7]))
+                 : "memory");
+}
+__device__ __forceinline__ void bwd_store_bf16_16_packed(uint8_t* dst, int r, int c0, const uint32_t (&w)[8]) {
+  const uint32_t d = smem_u32(dst);
+#pragma unroll
+  for (int q = 0; q < 2; ++q)
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d + bf16_tile_chunk(r, c0 + q)), "r"(w[4 * q]),
+                 "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
+                 : "memory");
+}
+
 // Descriptors of the three operand forms (start address, LBO, SBO, 128-byte
 // swizzle), with the per-step start-address advance of a K step:
 //   E4M3 tile, K-major:     32 columns = 32 bytes per step (+2 in the >> 4 field);
@@ -266,10 +286,52 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const BwdParams p) {
 }
 
 // --------------------------------------------------------------------------
-// dK and dV: one CTA (one warpgroup) per (batch, kv head, key tile).
+// dK and dV: one CTA per (batch, kv head, key tile).
+//
+// Roles: a TMA/MMA warp (warp 16, lane 0 issues) and two pairs of
+// warpgroups.  Pair p owns query half p (queries 64 p .. 64 p + 63) of every
+// step (query tile), with its own S^T / dP^T buffers in tensor memory (64
+// columns each), its own panel of the P^ and dS^T tiles and its own half of
+// Q's bfloat16 copy; within a pair, thread (key r, chunk c) takes 32 of the
+// half's 64 queries.  The MMA warp issues, for each step, each half's
+// products in a fixed order (so dV and dK sum in a fixed order): S^T and dP^T
+// of a half as soon as its inputs have landed, dV and dK of a half as soon as
+// its pair has written P^ and dS^T.  While one pair computes, the tensor core
+// works for the other.
 // --------------------------------------------------------------------------
-__global__ void __launch_bounds__(128 * kBwdGroups, 1)
-    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+constexpr int kDkdvCompute = 512;                 // two pairs of warpgroups
+constexpr int kDkdvThreads = kDkdvCompute + 32;   // + the TMA/MMA warp
+
+struct DkdvBars {
+  uint64_t kv;           // K_j and V_j landed
+  uint64_t q[2];         // Q half p of the step landed
+  uint64_t dout[2];      // dO of the step landed, one barrier per buffer (step parity)
+  uint64_t s_full[2];    // S^T and dP^T of half p computed
+  uint64_t qb_ready[2];  // pair p has converted its half of Q to bfloat16 (256 arrivals)
+  uint64_t p_full[2];    // pair p has written P^ and dS^T (256 arrivals)
+  uint64_t g_done[2];    // dV and dK products of half p complete
+  uint64_t drain;        // every product issued so far complete (end of the kernel)
+  uint32_t tmem_base;
+};
+
+// Pair-wide OR of `v` over the 256 threads of pair p (named barrier 1 + p).
+__device__ __forceinline__ bool pair_any(int p, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred a, b;\n\t"
+      "setp.ne.u32 a, %1, 0;\n\t"
+      "barrier.red.or.pred b, %2, 256, a;\n\t"
+      "selp.u32 %0, 1, 0, b;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "r"(1 + p)
+      : "memory");
+  return r != 0;
+}
+
+static_assert(sizeof(DkdvBars) <= 192, "dK/dV control block exceeds its shared-memory slot");
+
+__global__ void __launch_bounds__(kDkdvThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const BwdParams p, uint32_t* err_word) {
   using L = DkdvLayout;
@@ -277,210 +339,255 @@ __global__ void __launch_bounds__(128 * kBwdGroups, 1)
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* sLse2 = reinterpret_cast<float*>(base + L::OFF_VEC);
   float* sDelta = sLse2 + 128;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
-  uint64_t* bar_kv = bars + 0;     // K_j and V_j landed
-  uint64_t* bar_q = bars + 1;      // Q_i landed
-  uint64_t* bar_do = bars + 2;     // dO_i landed, one barrier per buffer (step parity)
-  uint64_t* bar_s = bars + 4;      // S^T and dP^T computed
-  uint64_t* bar_g = bars + 5;      // dV and dK products of this step complete
-  uint64_t* bar_drain = bars + 6;  // every product issued so far complete (abort path)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
+  DkdvBars* bars = reinterpret_cast<DkdvBars*>(base + L::OFF_BAR);
 
-  // kBwdGroups warpgroups: thread tid owns TMEM lane (key row) r = tid % 128
-  // and, in each step, part wg = tid / 128 of the queries (kBwdChunks chunks
-  // of 32).
-  const int tid = threadIdx.x, warp = tid >> 5, wg = tid >> 7, r = tid & 127;
+  const int tid = threadIdx.x, warp = tid >> 5;
   const int jt = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int k0 = jt * 128;
   const int zkv = b * p.Hkv + hk;
   const int i_first = p.causal ? jt : 0;  // query tiles before the key tile see none of its keys
   const int per_head = p.num_tiles - i_first;
   const int n_iter = p.h_per_kv * per_head;
-
-  if (tid == 0) {
-    for (int i = 0; i < 7; ++i) mbar_init(bars + i, 1);
-    fence_mbar_init();
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-    tma_prefetch_desc(&tm_do);
-  }
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, BwdConfig::TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tDP = tmem + 128, tDV = tmem + 256, tDK = tmem + 384;
-  const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-
   auto step_geom = [&](int it, int& zq, int& q0) {
     const int hl = it / per_head;
     q0 = (i_first + (it - hl * per_head)) * 128;
     zq = b * p.H + hk * p.h_per_kv + hl;
   };
-  // Thread 0's loads.  Q_i has one buffer: step it + 1's is fetched once
-  // S^T(it) is complete (Q(it) is already converted by then).  dO has two:
-  // step it + 2's goes to step it's buffer once step it's products are
-  // complete.  Issued / waited counts drive the drain after an abort.
-  int q_issued = 0, q_landed = 0, do_issued = 0, do_landed = 0;
-  auto issue_q = [&](int it) {
+
+  if (tid == kDkdvCompute) {
+    mbar_init(&bars->kv, 1);
+    mbar_init(&bars->drain, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->q[i], 1);
+      mbar_init(&bars->dout[i], 1);
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->qb_ready[i], 256);
+      mbar_init(&bars->p_full[i], 256);
+      mbar_init(&bars->g_done[i], 1);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q64);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_do);
+  }
+  if (warp == 0) {
+    tmem_alloc(&bars->tmem_base, BwdConfig::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  const uint32_t tDV = tmem + 256, tDK = tmem + 384;  // S^T / dP^T of half p at 128 p / 128 p + 64
+
+  // Loads (lane 0 of the MMA warp).
+  auto issue_q_half = [&](int it, int h) {
     int zq, q0;
     step_geom(it, zq, q0);
-    ++q_issued;
-    mbar_arrive_expect_tx(bar_q, BwdConfig::F8_TILE);
-    tma_load_3d(base + L::OFF_Q, &tm_q, bar_q, 0, q0, zq);
+    mbar_arrive_expect_tx(&bars->q[h], BwdConfig::F8_TILE / 2);
+    tma_load_3d(base + L::OFF_Q + h * (BwdConfig::F8_TILE / 2), &tm_q64, &bars->q[h], 0, q0 + 64 * h, zq);
   };
   auto issue_do = [&](int it) {
     int zq, q0;
     step_geom(it, zq, q0);
-    ++do_issued;
     uint8_t* dst = base + L::OFF_DO + (it & 1) * BwdConfig::BF_TILE;
-    mbar_arrive_expect_tx(bar_do + (it & 1), BwdConfig::BF_TILE);
-    tma_load_3d(dst, &tm_do, bar_do + (it & 1), 0, q0, zq);
-    tma_load_3d(dst + BwdConfig::BF_PANEL, &tm_do, bar_do + (it & 1), 64, q0, zq);
+    mbar_arrive_expect_tx(&bars->dout[it & 1], BwdConfig::BF_TILE);
+    tma_load_3d(dst, &tm_do, &bars->dout[it & 1], 0, q0, zq);
+    tma_load_3d(dst + BwdConfig::BF_PANEL, &tm_do, &bars->dout[it & 1], 64, q0, zq);
   };
-  if (tid == 0) {
+  if (tid == kDkdvCompute) {
     // V_j (E4M3) lands in the Q buffer, to be converted once.
-    mbar_arrive_expect_tx(bar_kv, 2 * BwdConfig::F8_TILE);
-    tma_load_3d(base + L::OFF_K, &tm_k, bar_kv, 0, k0, zkv);
-    tma_load_3d(base + L::OFF_Q, &tm_v, bar_kv, 0, k0, zkv);
+    mbar_arrive_expect_tx(&bars->kv, 2 * BwdConfig::F8_TILE);
+    tma_load_3d(base + L::OFF_K, &tm_k, &bars->kv, 0, k0, zkv);
+    tma_load_3d(base + L::OFF_Q, &tm_v, &bars->kv, 0, k0, zkv);
     if (n_iter > 0) issue_do(0);
     if (n_iter > 1) issue_do(1);
   }
+  bool fail = false;
+  if (tid < kDkdvCompute) {
+    fail = !mbar_wait_bounded(&bars->kv, 0, err_word, kErrTimeoutKV);
+    if (!fail) bwd_convert_part_row<2>(base + L::OFF_Q, base + L::OFF_VB, tid & 127, tid >> 7);
+    fence_proxy_async_smem();  // every thread has read V out of the Q buffer before Q may overwrite it
+  }
+  bool abort = __syncthreads_or(fail) != 0;
 
   const uint32_t sK = smem_u32(base + L::OFF_K), sVB = smem_u32(base + L::OFF_VB);
   const uint32_t sQ = smem_u32(base + L::OFF_Q), sQB = smem_u32(base + L::OFF_QB);
   const uint32_t sPT = smem_u32(base + L::OFF_PT), sDST = smem_u32(base + L::OFF_DST);
-  constexpr uint32_t idesc_s = idesc_e4m3_f32(128, 128, false, false);      // S^T = K Q^T
-  constexpr uint32_t idesc_dp = bwd_idesc_bf16(128, 128, false, false);     // dP^T = V dO^T
-  constexpr uint32_t idesc_grad = bwd_idesc_bf16(128, 128, false, true);    // dV += P^T dO, dK += dS^T Q
+  const uint32_t sDO0 = smem_u32(base + L::OFF_DO);
+  int q_issued[2] = {0, 0}, q_landed[2] = {0, 0}, do_issued = n_iter > 1 ? 2 : n_iter, do_landed = 0;
 
-  const int key = k0 + r;  // this thread's TMEM lane: one key
-  bool fail = !mbar_wait_bounded(bar_kv, 0, err_word, kErrTimeoutKV);
-  if (!fail) bwd_convert_part_row<8 / kBwdGroups>(base + L::OFF_Q, base + L::OFF_VB, r, wg);
-  // Every thread has read V out of the Q buffer before Q_0 may overwrite it.
-  fence_proxy_async_smem();
-  bool abort = __syncthreads_or(fail) != 0;
-  if (!abort && tid == 0 && n_iter > 0) issue_q(0);
-  // lse (warpgroup 0) and D (warpgroup 1) of the step's 128 queries, fetched
-  // one step ahead (the other warpgroups fetch nothing).
-  auto fetch_vec = [&](int it) -> float {
-    float x = 0.0f;
-    if (it < n_iter && wg < 2) {
-      int zq, q0;
-      step_geom(it, zq, q0);
-      const int qi = q0 + r;
-      if (qi < p.N) {
-        const int64_t idx = static_cast<int64_t>(zq) * p.N + qi;
-        x = (wg & 1) == 0 ? p.lse[idx] : p.delta[idx];  // used one step later
-      }
-    }
-    return x;
-  };
-  float next_vec = fetch_vec(0);
-
-  for (int it = 0; !abort && it < n_iter; ++it) {
-    if (wg == 0) sLse2[r] = next_vec * 1.4426950408889634f;  // lse in log2 units
-    if (wg == 1) sDelta[r] = next_vec;
-    next_vec = fetch_vec(it + 1);
-    const uint32_t sDO = smem_u32(base + L::OFF_DO + (it & 1) * BwdConfig::BF_TILE);
-    int zq, q0;
-    step_geom(it, zq, q0);
-    if (!fail && !mbar_wait_bounded(bar_q, it & 1, err_word, kErrTimeoutQ)) fail = true;
-    if (!fail && tid == 0) q_landed = it + 1;
-    if (!fail && !mbar_wait_bounded(bar_do + (it & 1), (it >> 1) & 1, err_word, kErrTimeoutQ)) fail = true;
-    if (!fail && tid == 0) do_landed = it + 1;
-    if (!fail) bwd_convert_part_row<8 / kBwdGroups>(base + L::OFF_Q, base + L::OFF_QB, r, wg);
-    fence_proxy_async_smem();
-    tc_fence_before();
-    abort = __syncthreads_or(fail) != 0;
-    if (abort) break;
-
-    if (tid == 0) {
+  if (tid == kDkdvCompute && !abort && n_iter > 0) {
+    // ----------------------------- TMA / MMA lane -----------------------------
+    constexpr uint32_t idesc_s = idesc_e4m3_f32(128, 64, false, false);   // S^T = K Q_h^T (N = 64 queries)
+    constexpr uint32_t idesc_dp = bwd_idesc_bf16(128, 64, false, false);  // dP^T = V dO_h^T
+    constexpr uint32_t idesc_grad = bwd_idesc_bf16(128, 128, false, true);  // dV += P^T dO_h, dK += dS^T Q_h
+    auto q_half = [&](int it, int h) {
+      issue_q_half(it, h);
+      ++q_issued[h];
+    };
+    // S^T and dP^T of half h of step it, once Q_h and dO of the step have landed.
+    auto issue_sdp = [&](int it, int h) -> bool {
+      if (!mbar_wait_bounded(&bars->q[h], it & 1, err_word, kErrTimeoutQ)) return false;
+      q_landed[h] = it + 1;
+      if (!mbar_wait_bounded(&bars->dout[it & 1], (it >> 1) & 1, err_word, kErrTimeoutQ)) return false;
+      do_landed = it + 1;
       tc_fence_after();
+      const uint32_t tS = tmem + 128 * h, tDP = tS + 64;
+      const uint32_t sQh = sQ + h * (BwdConfig::F8_TILE / 2);
+      const uint32_t sDOh = sDO0 + (it & 1) * BwdConfig::BF_TILE + h * (BwdConfig::BF_PANEL / 2);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_f8_ss(tS, kmajor_desc(sK) + 2 * kk, kmajor_desc(sQ) + 2 * kk, idesc_s, kk > 0);
+      for (int kk = 0; kk < 4; ++kk) mma_f8_ss(tS, kmajor_desc(sK) + 2 * kk, kmajor_desc(sQh) + 2 * kk, idesc_s, kk > 0);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        mma_bf16_ss(tDP, kmajor_desc(sVB) + bf16_kmajor_step(kk), kmajor_desc(sDO) + bf16_kmajor_step(kk),
-                    idesc_dp, kk > 0);
-      mma_commit(bar_s);
-    }
-    if (!mbar_wait_bounded(bar_s, it & 1, err_word, kErrTimeoutMMA)) fail = true;
-    tc_fence_after();
-    // S^T(it) has read Q(it), which is converted already: fetch the next Q.
-    if (tid == 0 && !fail && it + 1 < n_iter) issue_q(it + 1);
-
-    // P^T, E4M3(P^T S) and dS^T for this thread's key and its part of the
-    // queries, 32 at a time.
-    // Only tiles on the diagonal or past N mask any (key, query) pair.
-    const bool edge = q0 + 128 > p.N || k0 + 128 > p.N || (p.causal && k0 + 127 > q0);
-#pragma unroll 1
-    for (int g = kBwdChunks * wg; g < kBwdChunks * (wg + 1); ++g) {
-      uint32_t rs[32], rdp[32];
-      tmem_ld32(tS + lane_off + 32 * g, rs);
-      tmem_ld32(tDP + lane_off + 32 * g, rdp);
-      tmem_wait_ld();
-      uint32_t php[16];
-      float ds[32];
-#pragma unroll
-      for (int e4 = 0; e4 < 8; ++e4) {
-        const float4 lv = reinterpret_cast<const float4*>(sLse2 + 32 * g)[e4];
-        const float4 dv = reinterpret_cast<const float4*>(sDelta + 32 * g)[e4];
-        const float la[4] = {lv.x, lv.y, lv.z, lv.w}, da[4] = {dv.x, dv.y, dv.z, dv.w};
-        float pr[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int e = 4 * e4 + i;
-          pr[i] = ex2_approx(__uint_as_float(rs[e]) * p.scale_log2 - la[i]);
-          if (edge) {
-            const int qi = q0 + 32 * g + e;
-            const bool visible = qi < p.N && key < p.N && (!p.causal || key <= qi);
-            pr[i] = visible ? pr[i] : 0.0f;
-          }
-          ds[e] = pr[i] * (__uint_as_float(rdp[e]) - da[i]);
+        mma_bf16_ss(tDP, kmajor_desc(sVB) + bf16_kmajor_step(kk), kmajor_desc(sDOh) + bf16_kmajor_step(kk), idesc_dp,
+                    kk > 0);
+      mma_commit(&bars->s_full[h]);
+      return true;
+    };
+    q_half(0, 0);
+    q_half(0, 1);
+    bool ok = issue_sdp(0, 0) && issue_sdp(0, 1);
+    for (int it = 0; ok && it < n_iter; ++it) {
+      // dO of step it + 1 goes to the buffer of step it - 1 once both halves' products of that step completed.
+      if (it >= 1 && it + 1 < n_iter) {
+        ok = mbar_wait_bounded(&bars->g_done[0], (it - 1) & 1, err_word, kErrTimeoutMMA) &&
+             mbar_wait_bounded(&bars->g_done[1], (it - 1) & 1, err_word, kErrTimeoutMMA);
+        if (!ok) break;
+        issue_do(it + 1);
+        do_issued = it + 2;
+      }
+      // Q half h of step it + 1 once S^T(h, it) has completed and pair h has converted its half.
+      if (it + 1 < n_iter) {
+        for (int h = 0; ok && h < 2; ++h) {
+          ok = mbar_wait_bounded(&bars->s_full[h], it & 1, err_word, kErrTimeoutMMA) &&
+               mbar_wait_bounded(&bars->qb_ready[h], it & 1, err_word, kErrTimeoutPipe);
+          if (ok) q_half(it + 1, h);
         }
-        php[2 * e4] = bwd_e4m3_pair_bf16(pr[0] * p.p_scale, pr[1] * p.p_scale);
-        php[2 * e4 + 1] = bwd_e4m3_pair_bf16(pr[2] * p.p_scale, pr[3] * p.p_scale);
+        if (!ok) break;
       }
-      bwd_store_bf16_packed(base + L::OFF_PT, r, g, php);
-      bwd_store_bf16_32(base + L::OFF_DST, r, g, ds);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    abort = __syncthreads_or(fail) != 0;
-    if (abort) break;
-
-    if (tid == 0) {
-      tc_fence_after();
+      const uint32_t sDO = sDO0 + (it & 1) * BwdConfig::BF_TILE;
+      for (int h = 0; ok && h < 2; ++h) {
+        ok = mbar_wait_bounded(&bars->p_full[h], it & 1, err_word, kErrTimeoutPipe);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const bool acc = (it > 0) || (kk > 0);
-        mma_bf16_ss(tDV, kmajor_desc(sPT) + bf16_kmajor_step(kk), bf16_mnmajor_desc(sDO) + 128 * kk, idesc_grad,
-                    acc);
-        mma_bf16_ss(tDK, kmajor_desc(sDST) + bf16_kmajor_step(kk), bf16_mnmajor_desc(sQB) + 128 * kk,
-                    idesc_grad, acc);
+        for (int kk = 0; kk < 4; ++kk) {
+          const bool acc = (it > 0) || (h > 0) || (kk > 0);
+          const uint32_t rows = h * (BwdConfig::BF_PANEL / 2);  // queries 64 h .. of the MN-major operands
+          mma_bf16_ss(tDV, kmajor_desc(sPT + h * BwdConfig::BF_PANEL) + 2 * kk, bf16_mnmajor_desc(sDO + rows) + 128 * kk,
+                      idesc_grad, acc);
+          mma_bf16_ss(tDK, kmajor_desc(sDST + h * BwdConfig::BF_PANEL) + 2 * kk,
+                      bf16_mnmajor_desc(sQB + rows) + 128 * kk, idesc_grad, acc);
+        }
+        mma_commit(&bars->g_done[h]);
+        if (it + 1 < n_iter) ok = issue_sdp(it + 1, h);
       }
-      mma_commit(bar_g);
     }
-    if (!mbar_wait_bounded(bar_g, it & 1, err_word, kErrTimeoutMMA)) fail = true;
+    fail = !ok;
+  } else if (tid < kDkdvCompute && !abort) {
+    // ----------------------------- compute pairs ------------------------------
+    const int pr = tid >> 8, tp = tid & 255, c = tp >> 7, r = tid & 127;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + 128 * pr + lane_off, tDP = tS + 64;
+    const int key = k0 + r;
+    // lse (threads 0..63 of the pair) and D (64..127) of the pair's 64 queries, fetched one step ahead.
+    auto fetch = [&](int it) -> float {
+      if (it >= n_iter || tp >= 128) return 0.0f;
+      int zq, q0;
+      step_geom(it, zq, q0);
+      const int qi = q0 + 64 * pr + (tp & 63);
+      if (qi >= p.N) return 0.0f;
+      const int64_t idx = static_cast<int64_t>(zq) * p.N + qi;
+      return tp < 64 ? p.lse[idx] : p.delta[idx];
+    };
+    float next_vec = fetch(0);
+    for (int it = 0; it < n_iter; ++it) {
+      int zq, q0;
+      step_geom(it, zq, q0);
+      // This pair's previous products read P^, dS^T and its half of Q's bfloat16 copy.
+      if (it > 0 && !fail && !mbar_wait_bounded(&bars->g_done[pr], (it - 1) & 1, err_word, kErrTimeoutMMA))
+        fail = true;
+      if (tp < 64)
+        sLse2[64 * pr + tp] = next_vec * 1.4426950408889634f;  // lse in log2 units
+      else if (tp < 128)
+        sDelta[64 * pr + tp - 64] = next_vec;
+      next_vec = fetch(it + 1);
+      if (!fail && !mbar_wait_bounded(&bars->q[pr], it & 1, err_word, kErrTimeoutQ)) fail = true;
+      // Rows 64 pr .. 64 pr + 63 of Q to bfloat16, a quarter row per thread.
+      if (!fail) bwd_convert_part_row<2>(base + L::OFF_Q, base + L::OFF_QB, 64 * pr + (tp & 63), tp >> 6);
+      fence_proxy_async_smem();
+      mbar_arrive(&bars->qb_ready[pr]);
+      // One decision per pair (the barrier also makes the pair's lse/D writes visible).
+      if (pair_any(pr, fail)) {
+        fail = true;
+        break;
+      }
+      const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(&bars->s_full[pr], it & 1, err_word, kErrTimeoutMMA));
+      if (ok) {
+        tc_fence_after();
+        // P^T, E4M3(P^T S) and dS^T for this thread's key and queries 64 pr + 32 c .. + 31,
+        // 16 at a time (fewer live registers).
+        const int qh0 = q0 + 64 * pr;
+        const bool edge = qh0 + 64 > p.N || k0 + 128 > p.N || (p.causal && k0 + 127 > qh0);
+#pragma unroll 1
+        for (int sc = 0; sc < 2; ++sc) {
+          const int qc0 = 64 * pr + 32 * c + 16 * sc;  // first query column (in the tile) of the piece
+          uint32_t rs[16], rdp[16];
+          tmem_ld16(tS + 32 * c + 16 * sc, rs);
+          tmem_ld16(tDP + 32 * c + 16 * sc, rdp);
+          tmem_wait_ld();
+          uint32_t php[8];
+          float ds[16];
+#pragma unroll
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const float4 lv = reinterpret_cast<const float4*>(sLse2 + qc0)[e4];
+            const float4 dv = reinterpret_cast<const float4*>(sDelta + qc0)[e4];
+            const float la[4] = {lv.x, lv.y, lv.z, lv.w}, da[4] = {dv.x, dv.y, dv.z, dv.w};
+            float pb[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int e = 4 * e4 + i;
+              pb[i] = ex2_approx(__uint_as_float(rs[e]) * p.scale_log2 - la[i]);
+              if (edge) {
+                const int qi = q0 + qc0 + e;
+                const bool visible = qi < p.N && key < p.N && (!p.causal || key <= qi);
+                pb[i] = visible ? pb[i] : 0.0f;
+              }
+              ds[e] = pb[i] * (__uint_as_float(rdp[e]) - da[i]);
+            }
+            php[2 * e4] = bwd_e4m3_pair_bf16(pb[0] * p.p_scale, pb[1] * p.p_scale);
+            php[2 * e4 + 1] = bwd_e4m3_pair_bf16(pb[2] * p.p_scale, pb[3] * p.p_scale);
+          }
+          bwd_store_bf16_16_packed(base + L::OFF_PT, r, qc0 / 8, php);
+          bwd_store_bf16_16(base + L::OFF_DST, r, qc0 / 8, ds);
+        }
+        tc_fence_before();  // the loads of S^T / dP^T are ordered before p_full, which frees them
+      } else {
+        fail = true;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&bars->p_full[pr]);
+    }
+    // The last step's products of both halves.
+    if (!fail && n_iter > 0 &&
+        (!mbar_wait_bounded(&bars->g_done[0], (n_iter - 1) & 1, err_word, kErrTimeoutMMA) ||
+         !mbar_wait_bounded(&bars->g_done[1], (n_iter - 1) & 1, err_word, kErrTimeoutMMA)))
+      fail = true;
     tc_fence_after();
-    // This step's dO buffer is free again: fetch the dO of the step after next.
-    if (tid == 0 && !fail && it + 2 < n_iter) issue_do(it + 2);
   }
   abort = __syncthreads_or(fail || abort) != 0;
 
-  if (!abort) {
-    // Warpgroup 0 writes dV / S, warpgroup 1 dK / sqrt(d).  Every lane takes
-    // part in the warp-wide TMEM loads; lanes past N store nothing.
+  if (!abort && tid < kDkdvCompute) {
+    // dV / S and dK / sqrt(d): eight 32-column jobs, two per warpgroup.  Every
+    // lane takes part in the warp-wide TMEM loads; lanes past N store nothing.
+    const int wg = tid >> 7, r = tid & 127;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int key = k0 + r;
     const int64_t row = static_cast<int64_t>(zkv) * p.N + key;
-    // Jobs j = 0..7: dV chunks 0..3, then dK chunks 0..3, spread over the warpgroups.
 #pragma unroll 1
-    for (int job = wg * (8 / kBwdGroups); job < (wg + 1) * (8 / kBwdGroups); ++job) {
+    for (int job = 2 * wg; job < 2 * wg + 2; ++job) {
       const bool is_dv = job < 4;
       const int g = job & 3;
       float* dst = (is_dv ? p.dv : p.dk) + row * 128;
@@ -501,17 +608,21 @@ __global__ void __launch_bounds__(128 * kBwdGroups, 1)
         }
       }
     }
-  } else if (tid == 0) {
-    // A wait ran out: let the products and loads still in flight land before
-    // the CTA's tensor and shared memory are released (each wait again bounded).
-    mma_commit(bar_drain);
-    mbar_wait_bounded(bar_drain, 0, err_word, kErrTimeoutMMA, 100000000ull);
-    mbar_wait_bounded(bar_kv, 0, err_word, kErrTimeoutKV, 100000000ull);
-    for (int j = q_landed; j < q_issued; ++j) mbar_wait_bounded(bar_q, j & 1, err_word, kErrTimeoutQ, 100000000ull);
-    for (int j = do_landed; j < do_issued; ++j)
-      mbar_wait_bounded(bar_do + (j & 1), (j >> 1) & 1, err_word, kErrTimeoutQ, 100000000ull);
   }
-
+  if (tid == kDkdvCompute) {
+    // Every product issued has completed before tensor memory is released;
+    // after an abort, also the loads still in flight (each wait bounded).
+    mma_commit(&bars->drain);
+    mbar_wait_bounded(&bars->drain, 0, err_word, kErrTimeoutMMA, 100000000ull);
+    if (abort) {
+      mbar_wait_bounded(&bars->kv, 0, err_word, kErrTimeoutKV, 100000000ull);
+      for (int h = 0; h < 2; ++h)
+        for (int j = q_landed[h]; j < q_issued[h]; ++j)
+          mbar_wait_bounded(&bars->q[h], j & 1, err_word, kErrTimeoutQ, 100000000ull);
+      for (int j = do_landed; j < do_issued; ++j)
+        mbar_wait_bounded(&bars->dout[j & 1], (j >> 1) & 1, err_word, kErrTimeoutQ, 100000000ull);
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
