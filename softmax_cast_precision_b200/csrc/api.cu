@@ -689,7 +689,7 @@ extern "C" int fp8attn_quantize(const void* x, int x_dtype, void* xq, float* sca
   if (block_rows > 0 && static_cast<int64_t>(Z) * p.nblocks > (int64_t(1) << 30)) return FP8ATTN_ERR_UNSUPPORTED;
   p.x_f32 = x_dtype;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 128 ? launch_quantize<32>(p, s) : launch_quantize<16>(p, s);
+  return d == 128 ? launch_quantize<64>(p, s) : launch_quantize<32>(p, s);
 }
 
 extern "C" unsigned long long fp8attn_decode_workspace_bytes(int B, int H, int N, int split_tiles) {

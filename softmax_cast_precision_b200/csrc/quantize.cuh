@@ -13,13 +13,13 @@
 // engine at the block's amax barrier, when every thread has its rows in
 // registers.
 //
-// Four threads own one row.  The row is cut into 8-element chunks and thread
-// part t (0..3) holds chunks t, t + 4, t + 8, ... (E = d / 4 elements), so the
-// index of element i splits as i = 32 k + 8 t + j: j (bits 0-2) and k (bits
-// 5 and up) lie inside a thread, t (bits 3-4) across the row's four lanes.
+// Two adjacent lanes own one row.  The row is cut into 8-element chunks and
+// lane t (0, 1) of the pair holds chunks t, t + 2, t + 4, ... (E = d / 2
+// elements), so the index of element i splits as i = 16 m + 8 t + j: j (bits
+// 0-2) and m (bits 4 and up) lie inside a thread, t (bit 3) across the pair.
 // The rotation is the radix-2 fast transform with stages of half-width 1, 2,
 // ..., d/2, in that order (pair i, i + h: sum at i, difference at i + h):
-// half-widths 1, 2, 4 inside the thread, 8 and 16 through shuffles, 32 and 64
+// half-widths 1, 2, 4 inside the thread, 8 through one shuffle, 16 and up
 // inside the thread again.  Every operation rounds to float32 once, in that
 // fixed order.
 //
@@ -49,10 +49,10 @@ struct QuantParams {
 };
 
 constexpr int kQuantWarps = 8;
-constexpr int kQuantThreadsPerRow = 4;
-constexpr int kQuantRowsPerPass = kQuantWarps * 32 / kQuantThreadsPerRow;  // 64
+constexpr int kQuantThreadsPerRow = 2;
+constexpr int kQuantRowsPerPass = kQuantWarps * 32 / kQuantThreadsPerRow;  // 128: one block per pass
 constexpr int kQuantMaxStages = 8;
-constexpr int kQuantMaxChunks = 4;  // 8-element chunks per thread at d = 128
+constexpr int kQuantMaxChunks = 16;  // 8-element chunks per row at d = 128
 constexpr int kQuantStageBudget = 96 * 1024;  // shared bytes of the ring (two CTAs per SM)
 
 // Binary exponent e of the descale s = 2^e of a block whose largest
@@ -65,41 +65,44 @@ __device__ __forceinline__ int quant_scale_exponent(float amax) {
   return e < -126 ? -126 : e;
 }
 
-// One thread's E elements of a row, read from the staged block: slot c
-// (elements 8c .. 8c + 7 of the thread's list) holds chunk c ^ sw, row
-// elements 32 (c ^ sw) + 8 part ..  With sw = 1 on odd rows, the two rows of
-// a quarter-warp read opposite 64-byte halves of their 256-byte rows, so the
-// 16-byte reads hit distinct banks.  Rows past the block's end read as zeros.
+// One thread's E elements of a row, read from the staged block.  Thread t
+// (0, 1) of a row holds its chunks 2 m + t (8 elements each, m = 0 .. E/8 - 1):
+// slot k (elements 8 k .. 8 k + 7 of the thread's list) holds chunk
+// 2 (k ^ s) + t, where s = row % 4 for bfloat16 rows (0 otherwise), so the
+// four rows of a quarter-warp read distinct 16-byte banks.  Row element i
+// = 16 (k ^ s) + 8 t + j.  Rows past the block's end read as zeros.
 template <int E>
-__device__ __forceinline__ void quant_read_row(const uint8_t* stage, int row_bytes, int r, int rows, int part,
-                                               int x_f32, const uint4* sign_masks, int sw, float (&v)[E]) {
+__device__ __forceinline__ void quant_read_row(const uint8_t* stage, int row_bytes, int r, int rows, int t, int s,
+                                               int x_f32, const uint4* sign_masks, float (&v)[E]) {
   if (r >= rows) {
 #pragma unroll
     for (int e = 0; e < E; ++e) v[e] = 0.0f;
     return;
   }
   if (x_f32) {
-    const float* src = reinterpret_cast<const float*>(stage + static_cast<int64_t>(r) * row_bytes) + 8 * part;
+    const float* src = reinterpret_cast<const float*>(stage + static_cast<int64_t>(r) * row_bytes);
 #pragma unroll
-    for (int c = 0; c < E / 8; ++c) {
-      const float4 a = *reinterpret_cast<const float4*>(src + 32 * (c ^ sw));
-      const float4 b = *reinterpret_cast<const float4*>(src + 32 * (c ^ sw) + 4);
-      v[8 * c + 0] = a.x; v[8 * c + 1] = a.y; v[8 * c + 2] = a.z; v[8 * c + 3] = a.w;
-      v[8 * c + 4] = b.x; v[8 * c + 5] = b.y; v[8 * c + 6] = b.z; v[8 * c + 7] = b.w;
+    for (int k = 0; k < E / 8; ++k) {
+      const int c = 2 * (k ^ s) + t;
+      const float4 a = *reinterpret_cast<const float4*>(src + 8 * c);
+      const float4 b = *reinterpret_cast<const float4*>(src + 8 * c + 4);
+      v[8 * k + 0] = a.x; v[8 * k + 1] = a.y; v[8 * k + 2] = a.z; v[8 * k + 3] = a.w;
+      v[8 * k + 4] = b.x; v[8 * k + 5] = b.y; v[8 * k + 6] = b.z; v[8 * k + 7] = b.w;
     }
   } else {
     // bfloat16 -> float32 is exact: the 16 bits become the high half.
-    const uint16_t* src = reinterpret_cast<const uint16_t*>(stage + static_cast<int64_t>(r) * row_bytes) + 8 * part;
+    const uint16_t* src = reinterpret_cast<const uint16_t*>(stage + static_cast<int64_t>(r) * row_bytes);
 #pragma unroll
-    for (int c = 0; c < E / 8; ++c) {
-      const uint4 q = *reinterpret_cast<const uint4*>(src + 32 * (c ^ sw));
+    for (int k = 0; k < E / 8; ++k) {
+      const int c = 2 * (k ^ s) + t;
+      const uint4 q = *reinterpret_cast<const uint4*>(src + 8 * c);
       // With a rotation, the signs flip the bfloat16 sign bits (bits 15 and 31 of each word).
-      const uint4 sm = sign_masks ? sign_masks[(c ^ sw) * kQuantThreadsPerRow + part] : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 sm = sign_masks ? sign_masks[c] : make_uint4(0u, 0u, 0u, 0u);
       const uint32_t w[4] = {q.x ^ sm.x, q.y ^ sm.y, q.z ^ sm.z, q.w ^ sm.w};
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        v[8 * c + 2 * i] = __uint_as_float(w[i] << 16);
-        v[8 * c + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        v[8 * k + 2 * i] = __uint_as_float(w[i] << 16);
+        v[8 * k + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
       }
     }
   }
@@ -128,32 +131,34 @@ __device__ __forceinline__ void quant_stage(float (&v)[E]) {
   }
 }
 
-// The stage of half-width 32 (slot bit 0) when slots 2i and 2i + 1 may hold
-// chunks 2i + 1 and 2i (sw = 1): the member in slot 2i is then the upper
-// one.  new slot 2i = s1 * slot 2i + slot 2i+1, new slot 2i+1 = s2 * slot
-// 2i+1 + slot 2i, with (s1, s2) = (1, -1) or (-1, 1): a sum or a difference,
-// one rounding each, exactly as in the unswapped order.
-template <int E>
-__device__ __forceinline__ void quant_stage32(float (&v)[E], int sw) {
-  const float s1 = sw ? -1.0f : 1.0f;
+// An in-thread stage over a slot bit that s may flip: pairs (e, e + H) with
+// bit H of e clear; when flip is set, slot e holds the pair's upper member and
+// slot e + H its lower one.  Slot e becomes s1 v[e] + v[e + H] and slot e + H
+// becomes v[e] - s1 v[e + H] (s1 = -1 when flipped, else 1): the lower slot
+// gets the sum and the upper the difference, each rounded once, exactly as in
+// the unflipped order.
+template <int E, int H>
+__device__ __forceinline__ void quant_stage_flip(float (&v)[E], int flip) {
+  const float s1 = flip ? -1.0f : 1.0f;
   const uint64_t sg1 = f2_pack(s1, s1), sg2 = f2_pack(-s1, -s1);
 #pragma unroll
   for (int e = 0; e < E; e += 2) {
-    if ((e & 8) == 0) {
-      const uint64_t a = f2_pack(v[e], v[e + 1]), b = f2_pack(v[e + 8], v[e + 9]);
+    if ((e & H) == 0) {
+      const uint64_t a = f2_pack(v[e], v[e + 1]), b = f2_pack(v[e + H], v[e + 1 + H]);
       f2_unpack(f2_fma(a, sg1, b), v[e], v[e + 1]);
-      f2_unpack(f2_fma(b, sg2, a), v[e + 8], v[e + 9]);
+      f2_unpack(f2_fma(b, sg2, a), v[e + H], v[e + 1 + H]);
     }
   }
 }
 
 // The signs and the unnormalised transform x H_d over the thread's E values
-// (the factor 1/sqrt(d) is applied by the caller).  sb[c] holds the 8 sign
-// bits of chunk c (bit j set: element j of the chunk is negated); they are
-// applied here only when not already applied to the raw words (and then the
-// slots are not swapped, sw = 0).
+// (the factor 1/sqrt(d) is applied by the caller), stages of half-width 1, 2,
+// 4 inside the slots, 8 across the row's two threads, then 16, 32 (and 64)
+// over the slot bits.  sb[k] holds the 8 sign bits of slot k (bit j set:
+// element j is negated); they are applied here only when not already applied
+// to the raw words (and then s = 0).
 template <int E>
-__device__ __forceinline__ void quant_rotate_row(int part, const uint32_t (&sb)[E / 8], bool signs_applied, int sw,
+__device__ __forceinline__ void quant_rotate_row(int t, int s, const uint32_t (&sb)[E / 8], bool signs_applied,
                                                  float (&v)[E]) {
   if (!signs_applied) {
 #pragma unroll
@@ -164,43 +169,59 @@ __device__ __forceinline__ void quant_rotate_row(int part, const uint32_t (&sb)[
   quant_stage<E, 1>(v);
   quant_stage<E, 2>(v);
   quant_stage<E, 4>(v);
-  // Half-widths 8 and 16: the partner of element i is i ^ h, in lane part ^ (h / 8)
-  // at the same position; the lower member keeps v + other, the upper other - v.
-#pragma unroll
-  for (int hp = 1; hp < kQuantThreadsPerRow; hp *= 2) {
-    const float sg = (part & hp) ? -1.0f : 1.0f;
+  // Half-width 8: the partner of element i is i ^ 8, in the row's other
+  // thread at the same position; the lower member keeps v + other, the upper
+  // other - v.
+  {
+    const float sg = t ? -1.0f : 1.0f;
     const uint64_t sg2 = f2_pack(sg, sg);
 #pragma unroll
     for (int e = 0; e < E; e += 2) {
-      const float o0 = __shfl_xor_sync(0xffffffffu, v[e], hp);
-      const float o1 = __shfl_xor_sync(0xffffffffu, v[e + 1], hp);
+      const float o0 = __shfl_xor_sync(0xffffffffu, v[e], 1);
+      const float o1 = __shfl_xor_sync(0xffffffffu, v[e + 1], 1);
       f2_unpack(f2_fma(f2_pack(v[e], v[e + 1]), sg2, f2_pack(o0, o1)), v[e], v[e + 1]);
     }
   }
-  // Half-widths 32 and 64: chunk bits of the thread's list (8 and 16 in it).
-  quant_stage32<E>(v, sw);
-  if constexpr (E > 16) quant_stage<E, 16>(v);
+  // Half-widths 16, 32, 64: slot bits 0, 1, 2 (8, 16, 32 in the list); s flips bits 0 and 1.
+  quant_stage_flip<E, 8>(v, s & 1);
+  quant_stage_flip<E, 16>(v, (s >> 1) & 1);
+  if constexpr (E > 32) quant_stage<E, 32>(v);
 }
 
 // Stores E4M3(v * mul): mul = c / s, with c = float32(1/sqrt(d)) after a
 // rotation (else 1) and s the block's power-of-two descale, so that
-// v * mul = (v * c) / s exactly (s is a power of two).  Slot c (chunk c ^ sw)
-// goes to row bytes 32 (c ^ sw) + 8 part .. + 7.
+// v * mul = (v * c) / s exactly (s is a power of two).  Slot k holds chunk
+// 2 (k ^ sx) + t, row bytes 8 (2 (k ^ sx) + t) .. + 7; the two lanes of the
+// row swap half their slots so that each stores whole 16-byte pieces.  Every
+// lane calls this (the swap is a full-warp shuffle); `live` says whether the
+// row exists.
 template <int E>
-__device__ __forceinline__ void quant_store_row(uint8_t* dst_row, int part, const float (&v)[E], float mul, int sw) {
+__device__ __forceinline__ void quant_store_row(uint8_t* dst_row, bool live, int t, int sx, const float (&v)[E],
+                                                float mul) {
   const uint64_t m2 = f2_pack(mul, mul);
+  uint2 w[E / 8];
 #pragma unroll
-  for (int c = 0; c < E / 8; ++c) {
-    uint32_t w[2];
+  for (int k = 0; k < E / 8; ++k) {
+    float a, b, cc, dd;
+    f2_unpack(f2_mul(f2_pack(v[8 * k], v[8 * k + 1]), m2), a, b);
+    f2_unpack(f2_mul(f2_pack(v[8 * k + 2], v[8 * k + 3]), m2), cc, dd);
+    w[k].x = cvt_e4m3x4(a, b, cc, dd);
+    f2_unpack(f2_mul(f2_pack(v[8 * k + 4], v[8 * k + 5]), m2), a, b);
+    f2_unpack(f2_mul(f2_pack(v[8 * k + 6], v[8 * k + 7]), m2), cc, dd);
+    w[k].y = cvt_e4m3x4(a, b, cc, dd);
+  }
+  // Slots 2 q and 2 q + 1: lane t keeps slot 2 q + t and takes the partner's
+  // slot 2 q + t, which holds the other half of the same 16 bytes (chunks
+  // 2 m and 2 m + 1, m = (2 q + t) ^ sx), so that each lane stores 16 bytes.
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int e = 8 * c + 4 * j;
-      float a, b, cc, dd;
-      f2_unpack(f2_mul(f2_pack(v[e], v[e + 1]), m2), a, b);
-      f2_unpack(f2_mul(f2_pack(v[e + 2], v[e + 3]), m2), cc, dd);
-      w[j] = cvt_e4m3x4(a, b, cc, dd);
-    }
-    *reinterpret_cast<uint2*>(dst_row + 32 * (c ^ sw) + 8 * part) = make_uint2(w[0], w[1]);
+  for (int q = 0; q < E / 16; ++q) {
+    const uint2 mine = t ? w[2 * q + 1] : w[2 * q];
+    const uint2 give = t ? w[2 * q] : w[2 * q + 1];
+    uint2 got;
+    got.x = __shfl_xor_sync(0xffffffffu, give.x, 1);
+    got.y = __shfl_xor_sync(0xffffffffu, give.y, 1);
+    const uint4 out = t ? make_uint4(got.x, got.y, mine.x, mine.y) : make_uint4(mine.x, mine.y, got.x, got.y);
+    if (live) *reinterpret_cast<uint4*>(dst_row + 16 * ((2 * q + t) ^ sx)) = out;
   }
 }
 
@@ -226,12 +247,12 @@ __global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const Qua
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ __align__(8) uint64_t full[kQuantMaxStages];
   __shared__ float warp_amax[2][kQuantWarps];
-  // bfloat16 inputs with a rotation: XOR masks of the signs, per (chunk, part),
-  // for the four 32-bit words (two elements each) of a chunk.
-  __shared__ uint4 sign_masks[kQuantMaxChunks * kQuantThreadsPerRow];
+  // bfloat16 inputs with a rotation: XOR masks of the signs, per 8-element
+  // chunk of the row, for the four 32-bit words (two elements each) of a chunk.
+  __shared__ uint4 sign_masks[kQuantMaxChunks];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int part = lane & (kQuantThreadsPerRow - 1);
-  const int rsub = threadIdx.x / kQuantThreadsPerRow;  // 0..63
+  const int t = lane & 1;                               // which chunks of the row: 2 m + t
+  const int rsub = threadIdx.x / kQuantThreadsPerRow;  // 0..127
   const int row_bytes = p.d * (p.x_f32 ? 4 : 2);
   const int stage_bytes = quant_stage_bytes(p);
   const int stages = quant_stages(p);
@@ -244,10 +265,10 @@ __global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const Qua
   }
   const bool word_signs = p.rotate && !p.x_f32;
   if (word_signs && threadIdx.x < (E / 8) * kQuantThreadsPerRow) {
-    const int c = threadIdx.x / kQuantThreadsPerRow, pt = threadIdx.x % kQuantThreadsPerRow;
+    const int c = threadIdx.x, wi = c >> 2;  // chunk c: row elements 8 c .. 8 c + 7
     // (no run-time index into the parameter array, which would copy it to local memory)
-    const uint32_t word = c == 0 ? p.sign_bits[0] : c == 1 ? p.sign_bits[1] : c == 2 ? p.sign_bits[2] : p.sign_bits[3];
-    const uint32_t x = (word >> (8 * pt)) & 0xFFu;  // elements 32 c + 8 pt + j, bit j
+    const uint32_t word = wi == 0 ? p.sign_bits[0] : wi == 1 ? p.sign_bits[1] : wi == 2 ? p.sign_bits[2] : p.sign_bits[3];
+    const uint32_t x = (word >> (8 * (c & 3))) & 0xFFu;  // elements 8 c + j, bit j
     uint32_t m[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) m[j] = (((x >> (2 * j)) & 1u) << 15) | (((x >> (2 * j + 1)) & 1u) << 31);
@@ -269,17 +290,17 @@ __global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const Qua
     for (int k = 0; k < stages; ++k) issue(k);
   }
 
-  // This thread's sign bits: chunk c covers row elements 32 c + 8 part .. + 7.
+  // This thread's sign bits for float32 rows (no slot rotation there): slot k
+  // holds chunk 2 k + t, row elements 16 k + 8 t .. + 7, in sign word k / 2.
   uint32_t sb[E / 8];
 #pragma unroll
-  for (int c = 0; c < E / 8; ++c) sb[c] = (p.sign_bits[c] >> (8 * part)) & 0xFFu;
+  for (int k = 0; k < E / 8; ++k) sb[k] = (p.sign_bits[k >> 1] >> (8 * ((2 * k + t) & 3))) & 0xFFu;
   // float32(1/sqrt(d)) after a rotation: applied to the block maximum here
   // (positive scaling is monotone, so max |v c| = max|v| c) and folded into
   // the cast's multiplier.
-  const float cnorm = p.rotate ? ((E == 32) ? 0.08838834764831845f : 0.125f) : 1.0f;
-  // Odd rows hold their chunk pairs swapped (bfloat16 inputs; see quant_read_row).
-  // Every row this thread handles has the parity of rsub (rows rsub + 64 i).
-  const int sw = p.x_f32 ? 0 : (rsub & 1);
+  const float cnorm = p.rotate ? ((E == 64) ? 0.08838834764831845f : 0.125f) : 1.0f;
+  // Slot rotation of bfloat16 rows (see quant_read_row); the thread's row is rsub.
+  const int sx = p.x_f32 ? 0 : (rsub & 3);
 
   int k = 0;
   bool aborted = false;
@@ -290,17 +311,22 @@ __global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const Qua
     const bool ok = mbar_wait_bounded(&full[k % stages], (k / stages) & 1, err_word, kErrTimeoutLoad);
     const uint8_t* stage = ring + (k % stages) * stage_bytes;
     float v[kPasses][E];
-    float amax = 0.0f;
+    // Block maximum of |v| in four independent chains (max is exact in any order).
+    float am4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
     for (int i = 0; i < kPasses; ++i) {
       // Every lane transforms (rows past the block's end hold zeros), so the
       // full-warp shuffles of the rotation always have all 32 lanes.
-      quant_read_row<E>(stage, row_bytes, rsub + i * kQuantRowsPerPass, ok ? rows : 0, part, p.x_f32,
-                        word_signs ? sign_masks : nullptr, sw, v[i]);
-      if (p.rotate) quant_rotate_row<E>(part, sb, word_signs, sw, v[i]);
+      quant_read_row<E>(stage, row_bytes, rsub + i * kQuantRowsPerPass, ok ? rows : 0, t, sx, p.x_f32,
+                        word_signs ? sign_masks : nullptr, v[i]);
+      if (p.rotate) quant_rotate_row<E>(t, sx, sb, word_signs, v[i]);
 #pragma unroll
-      for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(v[i][e]));
+      for (int e = 0; e < E; e += 4) {
+        const float m01 = fmaxf(fabsf(v[i][e]), fabsf(v[i][e + 1])), m23 = fmaxf(fabsf(v[i][e + 2]), fabsf(v[i][e + 3]));
+        am4[(e / 4) & 3] = fmaxf(am4[(e / 4) & 3], fmaxf(m01, m23));
+      }
     }
+    float amax = fmaxf(fmaxf(am4[0], am4[1]), fmaxf(am4[2], am4[3]));
     if constexpr (MODE != 2) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
@@ -331,7 +357,8 @@ __global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const Qua
 #pragma unroll
     for (int i = 0; i < kPasses; ++i) {
       const int r = rsub + i * kQuantRowsPerPass;
-      if (r < rows) quant_store_row<E>(p.xq + (static_cast<int64_t>(z) * p.N + r0 + r) * p.d, part, v[i], mul, sw);
+      // (every lane takes part: the exchange inside is a full-warp shuffle)
+      quant_store_row<E>(p.xq + (static_cast<int64_t>(z) * p.N + r0 + r) * p.d, r < rows, t, sx, v[i], mul);
     }
   }
   // After a wait ran out: let the copies still in flight land before the CTA's
