@@ -200,8 +200,12 @@ unsigned long long fp8attn_decode_workspace_bytes(int B, int H, int N, int split
  * in float32.  The gradients do not depend on the forward call's kv_order.
  * d must be 128 (FP8ATTN_ERR_UNSUPPORTED otherwise); B * H * N at most 2^34.
  * All pointers are device pointers, caller-owned, 16-byte aligned (lse and
- * delta: 4-byte); the outputs are overwritten.  Allocates nothing; launches
- * three kernels on stream (the row dots, then dk and dv, then dq).
+ * delta: 4-byte); the outputs are overwritten, and no output may overlap
+ * another argument.  Allocates nothing: dk and dv also serve as scratch
+ * during the call (bfloat16 copies of k and v that the dq kernel reads,
+ * replaced by the gradients before the call's work ends).  Launches five
+ * kernels on stream: the row dots, the two bfloat16 copies, dq, then dk
+ * and dv.
  */
 int fp8attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                 const void* dout, float* dq, float* dk, float* dv, float* delta,

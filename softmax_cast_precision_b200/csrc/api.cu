@@ -782,10 +782,14 @@ extern "C" int fp8attn_bwd(const void* q, const void* k, const void* v, const vo
   p.p_scale = p_scale;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(128.0));
   p.inv_sqrt_d = static_cast<float>(1.0 / std::sqrt(128.0));
-  CUtensorMap tq, tq64, tk, tv, tdo;
+  // The dQ kernel reads bfloat16 copies of K and V, made into the dK and dV
+  // buffers (4 bytes per element; the copies take the first half) before the
+  // dK/dV kernel, which runs last, writes its results there.
+  CUtensorMap tq, tq64, tk, tv, tdo, tkb, tvb;
   if (!make_map(&tq, q, 128, N, B * H, 128) || !make_map(&tq64, q, 128, N, B * H, 64) ||
       !make_map(&tk, k, 128, N, B * Hkv, 128) || !make_map(&tv, v, 128, N, B * Hkv, 128) ||
-      !make_map_bf16(&tdo, dout, N, B * H))
+      !make_map_bf16(&tdo, dout, N, B * H) || !make_map_bf16(&tkb, dk, N, B * Hkv) ||
+      !make_map_bf16(&tvb, dv, N, B * Hkv))
     return FP8ATTN_ERR_CUDA;
   uint32_t* err_word = nullptr;
   if (cudaGetSymbolAddress(reinterpret_cast<void**>(&err_word), g_error_word) != cudaSuccess)
@@ -796,10 +800,17 @@ extern "C" int fp8attn_bwd(const void* q, const void* k, const void* v, const vo
           cudaSuccess)
     return FP8ATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int sms = num_sms();
+  if (sms <= 0) return FP8ATTN_ERR_CUDA;
   bwd_delta_kernel<<<static_cast<unsigned int>((rows + 7) / 8), 256, 0, s>>>(p);
+  const int64_t kv16 = static_cast<int64_t>(B) * Hkv * N * 8;  // 16-code groups of K (and of V)
+  const unsigned int widen_grid = static_cast<unsigned int>(std::min<int64_t>((kv16 + 255) / 256, 8LL * sms));
+  bwd_widen_kernel<<<widen_grid, 256, 0, s>>>(static_cast<const uint8_t*>(k), reinterpret_cast<uint16_t*>(dk), kv16);
+  bwd_widen_kernel<<<widen_grid, 256, 0, s>>>(static_cast<const uint8_t*>(v), reinterpret_cast<uint16_t*>(dv), kv16);
+  bwd_dq_kernel<<<dim3(p.num_tiles, H, B), 128 * kBwdGroups, DqLayout::SMEM_BYTES, s>>>(tq, tk, tkb, tvb, tdo, p,
+                                                                                     err_word);
   bwd_dkdv_kernel<<<dim3(p.num_tiles, Hkv, B), kDkdvThreads, DkdvLayout::SMEM_BYTES, s>>>(tq64, tk, tv, tdo, p,
                                                                                         err_word);
-  bwd_dq_kernel<<<dim3(p.num_tiles, H, B), 128 * kBwdGroups, DqLayout::SMEM_BYTES, s>>>(tq, tk, tv, tdo, p, err_word);
   return cudaGetLastError() == cudaSuccess ? FP8ATTN_OK : FP8ATTN_ERR_CUDA;
 }
 

@@ -13,8 +13,10 @@
 //
 // The cast is the identity for differentiation (dS uses the unquantised P).
 //
-// Three kernels, all on the caller's stream:
+// Four kernels, all on the caller's stream:
 //   bwd_delta_kernel  D_i = dO_i . O_i (one warp per row);
+//   bwd_widen_kernel  bfloat16 copies of K and V, written into the dK and dV
+//                     output buffers (free until bwd_dkdv_kernel writes them);
 //   bwd_dkdv_kernel   one CTA per (batch, kv head, 128-key tile): for every
 //                     query head of the group and every query tile that sees
 //                     the keys, S^T = K Q^T and dP^T = V dO^T on the tensor
@@ -23,13 +25,16 @@
 //                     tensor memory; no atomics (the group's heads are summed
 //                     in the CTA);
 //   bwd_dq_kernel     one CTA per (batch, head, 128-row query tile): S and dP
-//                     recomputed per key tile, dQ += dS K in tensor memory.
+//                     recomputed per key tile, dQ += dS K in tensor memory,
+//                     K and V loaded in bfloat16 from the widened copies;
+//                     it runs before bwd_dkdv_kernel, which overwrites them.
 //
 // Operands.  Q, K and V are E4M3 and dO is bfloat16.  S (S^T) multiplies two
 // E4M3 tiles (kind::f8f6f4).  The products with dO or dS take both operands
-// in bfloat16 (kind::f16): the E4M3 tiles are converted in shared memory,
-// exactly (every E4M3 value is a bfloat16 value), and so are the cast
-// probabilities E4M3(P S); dS is rounded to bfloat16 (nearest even).  Every
+// in bfloat16 (kind::f16): the E4M3 tiles are converted, exactly (every E4M3
+// value is a bfloat16 value) -- V and each Q tile in shared memory by the dK/dV
+// kernel, K and V once in global memory for the dQ kernel -- and so are the
+// cast probabilities E4M3(P S); dS is rounded to bfloat16 (nearest even).  Every
 // 16-bit tile is 128 rows x 128 columns stored as two 64-column panels under
 // the 128-byte swizzle (16 KB apart), the layout a TMA box of 64 bfloat16
 // columns writes; the MMAs read it K-major (K along the row) or MN-major (M
@@ -90,8 +95,7 @@ struct DqLayout {
   static constexpr int OFF_Q = 0;                                   // Q_i   E4M3
   static constexpr int OFF_DO = OFF_Q + BwdConfig::F8_TILE;         // dO_i  bf16
   static constexpr int OFF_K = OFF_DO + BwdConfig::BF_TILE;         // K_j   E4M3
-  static constexpr int OFF_V = OFF_K + BwdConfig::F8_TILE;          // V_j   E4M3
-  static constexpr int OFF_KB = OFF_V + BwdConfig::F8_TILE;         // K_j   bf16, two buffers (step parity)
+  static constexpr int OFF_KB = OFF_K + BwdConfig::F8_TILE;         // K_j   bf16, two buffers (step parity)
   static constexpr int OFF_VB = OFF_KB + 2 * BwdConfig::BF_TILE;    // V_j   bf16
   static constexpr int OFF_DS = OFF_VB + BwdConfig::BF_TILE;        // dS    bf16
   static constexpr int OFF_BAR = OFF_DS + BwdConfig::BF_TILE;
@@ -105,7 +109,7 @@ static_assert(DkdvLayout::OFF_VB % 1024 == 0 && DkdvLayout::OFF_Q % 1024 == 0 &&
                   DkdvLayout::OFF_QB % 1024 == 0 && DkdvLayout::OFF_DO % 1024 == 0 &&
                   DkdvLayout::OFF_PT % 1024 == 0 && DkdvLayout::OFF_DST % 1024 == 0,
               "dK/dV tiles must be 1024-byte aligned");
-static_assert(DqLayout::OFF_DO % 1024 == 0 && DqLayout::OFF_K % 1024 == 0 && DqLayout::OFF_V % 1024 == 0 &&
+static_assert(DqLayout::OFF_DO % 1024 == 0 && DqLayout::OFF_K % 1024 == 0 &&
                   DqLayout::OFF_KB % 1024 == 0 && DqLayout::OFF_VB % 1024 == 0 && DqLayout::OFF_DS % 1024 == 0,
               "dQ tiles must be 1024-byte aligned");
 static_assert(DkdvLayout::OFF_BAR % 8 == 0 && DqLayout::OFF_BAR % 8 == 0, "mbarriers are 8-byte aligned");
@@ -283,6 +287,20 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const BwdParams p) {
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
   if (lane == 0) p.delta[row] = s;
+}
+
+// E4M3 rows [n16 / 8][128] to bfloat16 rows [n16 / 8][128], 16 codes per
+// thread and step (exact, as in the shared-memory conversions).
+__global__ void __launch_bounds__(256) bwd_widen_kernel(const uint8_t* src, uint16_t* dst, int64_t n16) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 w = reinterpret_cast<const uint4*>(src)[i];
+    const uint2 a = bwd_e4m3x4_to_bf16x4(w.x), b = bwd_e4m3x4_to_bf16x4(w.y);
+    const uint2 c = bwd_e4m3x4_to_bf16x4(w.z), e = bwd_e4m3x4_to_bf16x4(w.w);
+    uint4* out = reinterpret_cast<uint4*>(dst) + 2 * i;
+    out[0] = make_uint4(a.x, a.y, b.x, b.y);
+    out[1] = make_uint4(c.x, c.y, e.x, e.y);
+  }
 }
 
 // --------------------------------------------------------------------------
@@ -636,14 +654,14 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
 // --------------------------------------------------------------------------
 __global__ void __launch_bounds__(128 * kBwdGroups, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                  const BwdParams p, uint32_t* err_word) {
+                  const __grid_constant__ CUtensorMap tm_kb, const __grid_constant__ CUtensorMap tm_vb,
+                  const __grid_constant__ CUtensorMap tm_do, const BwdParams p, uint32_t* err_word) {
   using L = DqLayout;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L::OFF_BAR);
   uint64_t* bar_q = bars + 0;   // Q_i and dO_i landed
-  uint64_t* bar_kv = bars + 1;  // K_j and V_j landed
+  uint64_t* bar_kv = bars + 1;  // K_j (E4M3 and bfloat16) and V_j (bfloat16) landed
   uint64_t* bar_s = bars + 2;   // S and dP computed
   uint64_t* bar_g = bars + 3;      // dQ product of this step complete
   uint64_t* bar_drain = bars + 4;  // every product issued so far complete (abort path)
@@ -665,7 +683,8 @@ __global__ void __launch_bounds__(128 * kBwdGroups, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_kb);
+    tma_prefetch_desc(&tm_vb);
     tma_prefetch_desc(&tm_do);
   }
   if (warp == 0) {
@@ -680,11 +699,17 @@ __global__ void __launch_bounds__(128 * kBwdGroups, 1)
   const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
 
   int kv_issued = 0, kv_landed = 0;  // thread 0: key tiles issued / waited for (drain after an abort)
+  // Key tile j: E4M3 K (for S), and bfloat16 K (for dQ, into buffer j % 2)
+  // and V (for dP) as two 64-column boxes each.
   auto issue_kv = [&](int j) {
     kv_issued = j + 1;
-    mbar_arrive_expect_tx(bar_kv, 2 * BwdConfig::F8_TILE);
+    mbar_arrive_expect_tx(bar_kv, BwdConfig::F8_TILE + 2 * BwdConfig::BF_TILE);
     tma_load_3d(base + L::OFF_K, &tm_k, bar_kv, 0, j * 128, zkv);
-    tma_load_3d(base + L::OFF_V, &tm_v, bar_kv, 0, j * 128, zkv);
+    uint8_t* kb = base + L::OFF_KB + (j & 1) * BwdConfig::BF_TILE;
+    tma_load_3d(kb, &tm_kb, bar_kv, 0, j * 128, zkv);
+    tma_load_3d(kb + BwdConfig::BF_PANEL, &tm_kb, bar_kv, 64, j * 128, zkv);
+    tma_load_3d(base + L::OFF_VB, &tm_vb, bar_kv, 0, j * 128, zkv);
+    tma_load_3d(base + L::OFF_VB + BwdConfig::BF_PANEL, &tm_vb, bar_kv, 64, j * 128, zkv);
   };
   if (tid == 0) {
     mbar_arrive_expect_tx(bar_q, BwdConfig::F8_TILE + BwdConfig::BF_TILE);
@@ -712,15 +737,6 @@ __global__ void __launch_bounds__(128 * kBwdGroups, 1)
     const int j0 = j * 128;
     if (!fail && !mbar_wait_bounded(bar_kv, j & 1, err_word, kErrTimeoutKV)) fail = true;
     if (!fail && tid == 0) kv_landed = j + 1;
-    if (!fail) {
-      // The first half of the warpgroups converts K, the second half V.
-      constexpr int kHalf = kBwdGroups / 2;
-      if (wg < kHalf)
-        bwd_convert_part_row<8 / kHalf>(base + L::OFF_K, base + L::OFF_KB + (j & 1) * BwdConfig::BF_TILE, r, wg);
-      else
-        bwd_convert_part_row<8 / kHalf>(base + L::OFF_V, base + L::OFF_VB, r, wg - kHalf);
-    }
-    fence_proxy_async_smem();
     tc_fence_before();
     abort = __syncthreads_or(fail) != 0;
     if (abort) break;
@@ -738,8 +754,9 @@ __global__ void __launch_bounds__(128 * kBwdGroups, 1)
     }
     if (!mbar_wait_bounded(bar_s, j & 1, err_word, kErrTimeoutMMA)) fail = true;
     tc_fence_after();
-    // The E4M3 K and V tiles have been read (S, and the conversions before
-    // the barrier): fetch the next key tile while this one is finished.
+    // S and dP have read K and V, and (the products of one thread completing
+    // in order) the dQ product of step j - 1 has read the other bfloat16 K
+    // buffer: fetch the next key tile while this one is finished.
     if (tid == 0 && !fail && j < last) issue_kv(j + 1);
 
     // Only tiles on the diagonal or past N mask any (query, key) pair.
