@@ -190,6 +190,19 @@ __device__ __forceinline__ void bwd_convert_part_row(const uint8_t* src, uint8_t
   }
 }
 
+// Shared-memory float stores and 16-byte loads by shared address.
+__device__ __forceinline__ void sts_f32(uint32_t addr, float x) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(x) : "memory");
+}
+__device__ __forceinline__ float4 lds_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
 // Stores 32 FP32 values (columns 32*g .. 32*g+31 of row `r`) as bfloat16
 // chunks 4g .. 4g+3 of a two-panel tile.
 __device__ __forceinline__ void bwd_store_bf16_32(uint8_t* dst, int r, int g, const float (&x)[32]) {
@@ -355,8 +368,9 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
   using L = DkdvLayout;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* sLse2 = reinterpret_cast<float*>(base + L::OFF_VEC);
-  float* sDelta = sLse2 + 128;
+  // lse_i * log2(e) and D_i of the step's queries; written and read through
+  // shared-memory addresses (generic pointers here would become generic loads).
+  const uint32_t sLse2 = smem_u32(base + L::OFF_VEC), sDelta = sLse2 + 128 * 4;
   DkdvBars* bars = reinterpret_cast<DkdvBars*>(base + L::OFF_BAR);
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -528,9 +542,9 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
       if (it > 0 && !fail && !mbar_wait_bounded(&bars->g_done[pr], (it - 1) & 1, err_word, kErrTimeoutMMA))
         fail = true;
       if (tp < 64)
-        sLse2[64 * pr + tp] = next_vec * 1.4426950408889634f;  // lse in log2 units
+        sts_f32(sLse2 + 4 * (64 * pr + tp), next_vec * 1.4426950408889634f);  // lse in log2 units
       else if (tp < 128)
-        sDelta[64 * pr + tp - 64] = next_vec;
+        sts_f32(sDelta + 4 * (64 * pr + tp - 64), next_vec);
       next_vec = fetch(it + 1);
       if (!fail && !mbar_wait_bounded(&bars->q[pr], it & 1, err_word, kErrTimeoutQ)) fail = true;
       // Rows 64 pr .. 64 pr + 63 of Q to bfloat16, a quarter row per thread.
@@ -560,8 +574,8 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
           float ds[16];
 #pragma unroll
           for (int e4 = 0; e4 < 4; ++e4) {
-            const float4 lv = reinterpret_cast<const float4*>(sLse2 + qc0)[e4];
-            const float4 dv = reinterpret_cast<const float4*>(sDelta + qc0)[e4];
+            const float4 lv = lds_f32x4(sLse2 + 4 * qc0 + 16 * e4);
+            const float4 dv = lds_f32x4(sDelta + 4 * qc0 + 16 * e4);
             const float la[4] = {lv.x, lv.y, lv.z, lv.w}, da[4] = {dv.x, dv.y, dv.z, dv.w};
             float pb[4];
 #pragma unroll
