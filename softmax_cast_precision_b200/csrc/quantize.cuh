@@ -48,7 +48,7 @@ struct QuantParams {
   uint32_t sign_bits[4];  // bit i set: signs[i] = -1 (d <= 128)
 };
 
-constexpr int kQuantWarps = 8;
+constexpr int kQuantWarps = 8;  // the block maximum reads the warps' maxima as two float4
 constexpr int kQuantThreadsPerRow = 2;
 constexpr int kQuantRowsPerPass = kQuantWarps * 32 / kQuantThreadsPerRow;  // 128: one block per pass
 constexpr int kQuantMaxStages = 8;
@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const Qua
   constexpr int kPasses = 128 / kQuantRowsPerPass;  // rows per thread held in registers (block_rows <= 128)
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ __align__(8) uint64_t full[kQuantMaxStages];
-  __shared__ float warp_amax[2][kQuantWarps];
+  __shared__ __align__(16) float warp_amax[2][kQuantWarps];
   // bfloat16 inputs with a rotation: XOR masks of the signs, per 8-element
   // chunk of the row, for the four 32-bit words (two elements each) of a chunk.
   __shared__ uint4 sign_masks[kQuantMaxChunks];
@@ -328,8 +328,7 @@ __global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const Qua
     }
     float amax = fmaxf(fmaxf(am4[0], am4[1]), fmaxf(am4[2], am4[3]));
     if constexpr (MODE != 2) {
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      amax = warp_max_f32(amax);
       if (lane == 0) warp_amax[k & 1][warp] = amax;
     }
     // Every thread holds its rows: the stage goes back to the copy engine.
@@ -342,9 +341,9 @@ __global__ void __launch_bounds__(kQuantWarps * 32, 2) quantize_kernel(const Qua
     if constexpr (MODE == 2) {
       e = quant_scale_exponent(__uint_as_float(reinterpret_cast<const uint32_t*>(p.scales)[z]));
     } else {
-      float a = warp_amax[k & 1][0];
-#pragma unroll
-      for (int w = 1; w < kQuantWarps; ++w) a = fmaxf(a, warp_amax[k & 1][w]);
+      const float4 w0 = reinterpret_cast<const float4*>(warp_amax[k & 1])[0];
+      const float4 w1 = reinterpret_cast<const float4*>(warp_amax[k & 1])[1];
+      float a = fmaxf(fmaxf(fmaxf(w0.x, w0.y), fmaxf(w0.z, w0.w)), fmaxf(fmaxf(w1.x, w1.y), fmaxf(w1.z, w1.w)));
       a *= cnorm;
       if constexpr (MODE == 1) {
         if (threadIdx.x == 0) atomicMax(reinterpret_cast<unsigned int*>(p.scales + z), __float_as_uint(a));
