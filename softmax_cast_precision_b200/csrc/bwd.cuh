@@ -563,7 +563,7 @@ __global__ void __launch_bounds__(kDkdvThreads, 1)
         // 16 at a time (fewer live registers).
         const int qh0 = q0 + 64 * pr;
         const bool edge = qh0 + 64 > p.N || k0 + 128 > p.N || (p.causal && k0 + 127 > qh0);
-#pragma unroll 1
+#pragma unroll
         for (int sc = 0; sc < 2; ++sc) {
           const int qc0 = 64 * pr + 32 * c + 16 * sc;  // first query column (in the tile) of the piece
           uint32_t rs[16], rdp[16];
