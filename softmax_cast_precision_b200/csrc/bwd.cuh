@@ -143,31 +143,9 @@ __device__ __forceinline__ uint2 bwd_e4m3x4_to_bf16x4(uint32_t w) {
   return make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(b.x, b.y));
 }
 
-// Row `r` of an E4M3 tile (128 bytes per row, 128-byte swizzle, as TMA wrote
-// it) into row `r` of a two-panel bfloat16 tile.
-__device__ __forceinline__ void bwd_convert_row(const uint8_t* src, uint8_t* dst, int r) {
-  const uint32_t s = smem_u32(src), d = smem_u32(dst);
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint32_t w0, w1, w2, w3;
-    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(w0), "=r"(w1), "=r"(w2), "=r"(w3)
-                 : "r"(s + r * 128 + ((c ^ (r & 7)) << 4))
-                 : "memory");
-    // 16 E4M3 columns 16c .. 16c+15 become bfloat16 chunks 2c and 2c+1.
-    const uint2 a = bwd_e4m3x4_to_bf16x4(w0), b = bwd_e4m3x4_to_bf16x4(w1);
-    const uint2 e = bwd_e4m3x4_to_bf16x4(w2), f = bwd_e4m3x4_to_bf16x4(w3);
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d + bf16_tile_chunk(r, 2 * c)), "r"(a.x),
-                 "r"(a.y), "r"(b.x), "r"(b.y)
-                 : "memory");
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d + bf16_tile_chunk(r, 2 * c + 1)), "r"(e.x),
-                 "r"(e.y), "r"(f.x), "r"(f.y)
-                 : "memory");
-  }
-}
-
-// Part h of that: E4M3 columns 16 NC h .. 16 NC (h + 1) - 1 of row `r`, so
-// that 8 / NC threads share the conversion of a row.
+// Part h of row `r` of an E4M3 tile (128 bytes per row, 128-byte swizzle, as
+// TMA wrote it) into row `r` of a two-panel bfloat16 tile: E4M3 columns
+// 16 NC h .. 16 NC (h + 1) - 1, so that 8 / NC threads share a row.
 template <int NC>
 __device__ __forceinline__ void bwd_convert_part_row(const uint8_t* src, uint8_t* dst, int r, int h) {
   const uint32_t s = smem_u32(src), d = smem_u32(dst);
@@ -227,17 +205,6 @@ __device__ __forceinline__ uint32_t bwd_e4m3_pair_bf16(float lo, float hi) {
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<uint16_t>(code)));
   const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
   return pack_bf16x2(f.x, f.y);
-}
-
-// Stores 32 values already packed as 16 bfloat16 pairs (columns 32 g ..
-// 32 g + 31 of row `r`) as chunks 4g .. 4g+3 of a two-panel tile.
-__device__ __forceinline__ void bwd_store_bf16_packed(uint8_t* dst, int r, int g, const uint32_t (&w)[16]) {
-  const uint32_t d = smem_u32(dst);
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(d + bf16_tile_chunk(r, 4 * g + q)), "r"(w[4 * q]),
-                 "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
-                 : "memory");
 }
 
 // 16 values (columns 8 c0 .. 8 c0 + 15 of row `r`) as bfloat16 chunks c0 and
